@@ -1,0 +1,189 @@
+// Host side of the tcgen05 GEMM: TMA tensor maps, tile-width choice, launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "aut_gemm.cuh"
+#include "aut_internal.h"
+#include "aut_kernels.h"
+
+namespace aut {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims innermost first, strides in bytes
+// for dims 1.., box in elements.  Out-of-range elements of a box read as zero.
+bool make_map(CUtensorMap *m, int rank, const void *ptr, const cuuint64_t *dims,
+              const cuuint64_t *strides, const cuuint32_t *box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(ptr), dims,
+              strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 1;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int BN>
+GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+               cudaStream_t st) {
+    using Cfg = GemmCfg<BN>;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return GemmStatus::kLaunch;
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES) != cudaSuccess)
+            return GemmStatus::kLaunch;
+        attr_done[dev] = true;
+    }
+    const int tiles = args.num_m_tiles * args.num_n_tiles;
+    const int grid = std::min(tiles, sm_count());
+    gemm_tc_kernel<BN><<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, args);
+    return cudaGetLastError() == cudaSuccess ? GemmStatus::kOk : GemmStatus::kLaunch;
+}
+
+GemmStatus dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+                    cudaStream_t st) {
+    switch (bn) {
+        case 16: return run<16>(ta, tb, args, st);
+        case 32: return run<32>(ta, tb, args, st);
+        case 64: return run<64>(ta, tb, args, st);
+        case 128: return run<128>(ta, tb, args, st);
+        case 192: return run<192>(ta, tb, args, st);
+        case 240: return run<240>(ta, tb, args, st);
+        case 256: return run<256>(ta, tb, args, st);
+        default: return GemmStatus::kBadShape;
+    }
+}
+
+// Tile width for a plain GEMM: the candidate that divides N with the fewest
+// (waves x per-tile cost); wider tiles reuse each A tile over more columns.
+int choose_bn(int M, int N, int sms) {
+    static const int cand[] = {256, 128, 64, 32, 16};
+    const int mt = (M + 127) / 128;
+    int best = 0;
+    long best_cost = 0;
+    for (int bn : cand) {
+        if (N % bn) continue;
+        const long tiles = (long)mt * (N / bn);
+        const long waves = (tiles + sms - 1) / sms;
+        const long cost = waves * (bn + 32);
+        if (!best || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+}  // namespace
+
+GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
+    if (L.M <= 0) return GemmStatus::kOk;
+    if (L.N <= 0 || L.K <= 0 || L.K % 64 || L.N % 16 || !L.a || !L.w || !L.out)
+        return GemmStatus::kBadShape;
+    if (!aligned16(L.a) || !aligned16(L.w) || !aligned16(L.out) || (L.bias && !aligned16(L.bias)))
+        return GemmStatus::kBadShape;
+    const int bn = choose_bn(L.M, L.N, sm_count());
+    if (!bn) return GemmStatus::kBadShape;
+    CUtensorMap ta, tb;
+    const cuuint64_t da[2] = {(cuuint64_t)L.K, (cuuint64_t)L.M};
+    const cuuint64_t sa[1] = {(cuuint64_t)L.K * 2};
+    const cuuint32_t ba[2] = {64, 128};
+    const cuuint64_t db[2] = {(cuuint64_t)L.K, (cuuint64_t)L.N};
+    const cuuint32_t bb[2] = {64, (cuuint32_t)bn};
+    if (!make_map(&ta, 2, L.a, da, sa, ba) || !make_map(&tb, 2, L.w, db, sa, bb))
+        return GemmStatus::kTensorMap;
+    GemmArgs args{};
+    args.M = L.M;
+    args.N = L.N;
+    args.num_m_tiles = (L.M + 127) / 128;
+    args.num_n_tiles = L.N / bn;
+    args.num_k_blocks = L.K / 64;
+    args.conv = 0;
+    args.epi = L.epi;
+    args.bias = static_cast<const __nv_bfloat16 *>(L.bias);
+    args.out = L.out;
+    args.ldo = L.ldo;
+    args.chunks = L.chunks;
+    args.chunk_base = L.chunk_base;
+    args.pos = L.pos;
+    args.status = L.status;
+    args.timeout_ns = L.timeout_ns;
+    args.fault_inject = L.fault_inject;
+    return dispatch(bn, ta, tb, args, st);
+}
+
+GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
+    if (L.chunks <= 0) return GemmStatus::kOk;
+    const int bn = conv_tile_n(L.C);
+    if (!bn || L.rows_per_tile * L.out_cols > 128) return GemmStatus::kBadShape;
+    if (!aligned16(L.planes) || !aligned16(L.w_tap) || !aligned16(L.out) || !aligned16(L.bias))
+        return GemmStatus::kBadShape;
+    const long rows_total = (long)L.chunks * L.chunk_rows;
+    CUtensorMap ta, tb;
+    const cuuint64_t da[4] = {(cuuint64_t)L.C, (cuuint64_t)L.cols_in, (cuuint64_t)rows_total, 4};
+    const cuuint64_t sa[3] = {(cuuint64_t)L.C * 2, (cuuint64_t)L.cols_in * L.C * 2,
+                              (cuuint64_t)L.plane_rows_cap * L.cols_in * L.C * 2};
+    const cuuint32_t ba[4] = {64, (cuuint32_t)L.out_cols, (cuuint32_t)L.rows_per_tile, 1};
+    const cuuint64_t db[3] = {(cuuint64_t)L.C, 9, (cuuint64_t)L.C};
+    const cuuint64_t sb[2] = {(cuuint64_t)L.C * 2, (cuuint64_t)9 * L.C * 2};
+    const cuuint32_t bb[3] = {64, 1, (cuuint32_t)bn};
+    if (!make_map(&ta, 4, L.planes, da, sa, ba) || !make_map(&tb, 3, L.w_tap, db, sb, bb))
+        return GemmStatus::kTensorMap;
+    GemmArgs args{};
+    args.M = (int)rows_total;
+    args.N = L.C;
+    args.num_m_tiles = (int)((rows_total + L.rows_per_tile - 1) / L.rows_per_tile);
+    args.num_n_tiles = L.C / bn;
+    args.conv = 1;
+    args.conv_rows = L.rows_per_tile;
+    args.conv_cols = L.out_cols;
+    args.conv_vrows = L.chunk_rows;
+    args.conv_cblocks = (L.C + 63) / 64;
+    args.conv_chunks = L.chunks;
+    args.num_k_blocks = 9 * args.conv_cblocks;
+    args.epi = L.epi;
+    args.bias = static_cast<const __nv_bfloat16 *>(L.bias);
+    args.out = L.out;
+    args.C = L.C;
+    args.dst_plane_rows = L.dst_plane_rows;
+    args.dst_chunk_rows = L.dst_chunk_rows;
+    args.dst_cols = L.dst_cols;
+    args.status = L.status;
+    args.timeout_ns = L.timeout_ns;
+    return dispatch(bn, ta, tb, args, st);
+}
+
+}  // namespace aut

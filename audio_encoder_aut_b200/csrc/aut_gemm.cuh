@@ -1,0 +1,395 @@
+// Persistent tcgen05 GEMM for sm_100a: D[M, N] = A[M, K] * B[N, K]^T (bf16 in,
+// fp32 accumulate in tensor memory) with fused epilogues.
+//
+// Every GEMM of the encoder runs through this kernel:
+//   - the linear layers (qkv_proj, o_proj, fc1, fc2, proj1, proj2) with bias,
+//     bias + GELU, or bias + residual add into the fp32 residual stream;
+//   - conv2 and conv3 of the stem as implicit GEMMs: the A operand of filter
+//     tap (kh, kw) is a plain rectangle of one stride-2 phase plane of the
+//     previous conv's output, so TMA loads it directly (no im2col buffer);
+//   - conv_out, whose epilogue adds the chunk's sinusoid row, drops the tokens
+//     past the chunk's valid length and writes each kept row to its packed
+//     position (token packing fused into the GEMM).
+//
+// Block = 6 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory
+// ring, warp 1 owns the tensor-memory allocation and issues tcgen05.mma from
+// one thread, warps 2-5 drain the accumulator (tcgen05.ld) and run the
+// epilogue.  Two accumulators in tensor memory let the epilogue of one tile
+// overlap the MMAs of the next.  Tiles are 128 x BN x 64 (bf16, 128-byte
+// swizzle); the grid is persistent (one CTA per SM, tiles strided by gridDim).
+// Every mbarrier wait is bounded: on time-out the kernel records
+// AUT_ERR_TIMEOUT in the status word, stops all roles, waits for its own copies
+// and MMAs in flight, frees tensor memory and returns.
+#pragma once
+
+#include "aut_kernels.h"
+#include "aut_ptx.cuh"
+
+namespace aut {
+
+constexpr int kTokensPerChunkDev = 13;  // tokens out of one 100-frame chunk
+
+// Epilogue codes (GemmEpilogue) are declared in aut_kernels.h.
+
+struct GemmArgs {
+    int M, N;
+    int num_m_tiles, num_n_tiles, num_k_blocks;
+    // implicit-GEMM convolution operand (conv = 1)
+    int conv;
+    int conv_rows;     // virtual plane rows per M tile
+    int conv_cols;     // output columns per virtual row
+    int conv_vrows;    // virtual rows per chunk: output rows + 1 spare
+    int conv_cblocks;  // 64-channel blocks per filter tap
+    int conv_chunks;   // chunks in this group
+    // epilogue
+    int epi;
+    const __nv_bfloat16 *bias;  // [N] or nullptr
+    void *out;
+    int ldo;
+    int C;               // conv channels (conv epilogues)
+    int dst_plane_rows;  // rows of one destination phase plane (kEpiConvPlanes)
+    int dst_chunk_rows;  // destination plane rows per chunk, zero row included
+    int dst_cols;        // destination plane columns, zero column included
+    const int4 *chunks;  // chunk records {request, frame0, valid_frames, token0}
+    int chunk_base;      // global index of the group's first chunk (kEpiPackTokens)
+    const float *pos;    // sinusoid table [13][N] or nullptr (kEpiPackTokens)
+    // failure reporting
+    int *status;
+    unsigned long long timeout_ns;
+    int fault_inject;
+};
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int BM = 128, BK = 64;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES_FIT = 196608 / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static constexpr int TMEM_COLS = (2 * BN <= 32)    ? 32
+                                     : (2 * BN <= 64)  ? 64
+                                     : (2 * BN <= 128) ? 128
+                                     : (2 * BN <= 256) ? 256
+                                                       : 512;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + BAR_BYTES;
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M = 128");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+};
+
+AUT_DEV void gemm_signal_abort(const GemmArgs &args, volatile int *abort_flag) {
+    if (args.status) atomicCAS(args.status, 0, kDevTimeout);
+    *abort_flag = 1;
+}
+
+AUT_DEV int stem_tokens_dev(int v) {
+    v = v > 0 ? (v + 1) / 2 : 0;
+    v = v > 0 ? (v + 1) / 2 : 0;
+    return v > 0 ? (v + 1) / 2 : 0;
+}
+
+// Converts 16 fp32 values to bf16 and stores them (32 contiguous bytes).
+AUT_DEV void store_bf16x16(__nv_bfloat16 *p, const float (&v)[16]) {
+    uint4 a, b;
+    a.x = pack_bf16x2(v[0], v[1]);
+    a.y = pack_bf16x2(v[2], v[3]);
+    a.z = pack_bf16x2(v[4], v[5]);
+    a.w = pack_bf16x2(v[6], v[7]);
+    b.x = pack_bf16x2(v[8], v[9]);
+    b.y = pack_bf16x2(v[10], v[11]);
+    b.z = pack_bf16x2(v[12], v[13]);
+    b.w = pack_bf16x2(v[14], v[15]);
+    reinterpret_cast<uint4 *>(p)[0] = a;
+    reinterpret_cast<uint4 *>(p)[1] = b;
+}
+
+AUT_DEV void add_bias16(float (&v)[16], const __nv_bfloat16 *bias, int n0) {
+    if (!bias) return;
+    const uint4 *bp = reinterpret_cast<const uint4 *>(bias + n0);
+    const uint4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
+    const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&b0);
+    const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&b1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f0 = __bfloat1622float2(h0[i]);
+        float2 f1 = __bfloat1622float2(h1[i]);
+        v[2 * i] += f0.x;
+        v[2 * i + 1] += f0.y;
+        v[8 + 2 * i] += f1.x;
+        v[8 + 2 * i + 1] += f1.y;
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs args) {
+    using Cfg = GemmCfg<BN>;
+    constexpr int STAGES = Cfg::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + STAGES * Cfg::A_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * Cfg::STAGE_BYTES);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *mma_done = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, 4);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    volatile int *abort_v = abort_flag;
+    const int total_tiles = args.num_m_tiles * args.num_n_tiles;
+    const uint64_t lim = args.timeout_ns;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer --
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, parity = 0;
+            bool ok = true, skip = args.fault_inject != 0 && blockIdx.x == 0;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+                const int n_blk = tile % args.num_n_tiles, m_blk = tile / args.num_n_tiles;
+                for (int kb = 0; kb < args.num_k_blocks; ++kb) {
+                    if (!mbar_wait(empty + stage, phase ^ 1u, abort_v, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    if (skip) {
+                        skip = false;  // injected fault: this stage is never filled
+                    } else {
+                        uint8_t *a_dst = sA + stage * Cfg::A_BYTES;
+                        uint8_t *b_dst = sB + stage * Cfg::B_BYTES;
+                        if (!args.conv) {
+                            mbar_arrive_expect_tx(full + stage, Cfg::A_BYTES + Cfg::B_BYTES);
+                            tma_load_2d(a_dst, &tmA, full + stage, kb * 64, m_blk * 128);
+                            tma_load_2d(b_dst, &tmB, full + stage, kb * 64, n_blk * BN);
+                        } else {
+                            const int tap = kb / args.conv_cblocks;
+                            const int cb = kb - tap * args.conv_cblocks;
+                            const int kh = tap / 3, kw = tap - 3 * (tap / 3);
+                            // tap kh reads input row 2i + kh - 1: phase 1 for kh in {0, 2},
+                            // phase 0 for kh = 1; plane row i (kh = 0) or i + 1 (kh = 1, 2)
+                            // counting the leading zero row.  Same for kw along columns.
+                            const int plane = (kh == 1 ? 0 : 2) + (kw == 1 ? 0 : 1);
+                            const int dh = kh == 0 ? 0 : 1, dw = kw == 0 ? 0 : 1;
+                            const uint32_t a_bytes = 128u * args.conv_rows * args.conv_cols;
+                            mbar_arrive_expect_tx(full + stage, a_bytes + Cfg::B_BYTES);
+                            tma_load_4d(a_dst, &tmA, full + stage, cb * 64, dw,
+                                        m_blk * args.conv_rows + dh, plane);
+                            tma_load_3d(b_dst, &tmB, full + stage, cb * 64, tap, n_blk * BN);
+                        }
+                        issued |= 1u << stage;
+                        parity = (parity & ~(1u << stage)) | (phase << stage);
+                    }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) gemm_signal_abort(args, abort_v);
+            // The last load issued on every stage has landed before the block may exit.
+            for (int s = 0; s < STAGES; ++s)
+                if (issued >> s & 1u) mbar_wait(full + s, parity >> s & 1u, nullptr, lim);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // -------------------------------------------------- MMA issuer --
+            constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+            int stage = 0, it = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(tempty + acc, acc_phase ^ 1u, abort_v, lim)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kb = 0; kb < args.num_k_blocks; ++kb) {
+                    if (!mbar_wait(full + stage, phase, abort_v, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = smem_desc_sw128(sA + stage * Cfg::A_BYTES);
+                    const uint64_t b_desc = smem_desc_sw128(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // K = 16 per MMA: +32 bytes in the row
+                        tc_mma_bf16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
+                                    (kb | kk) != 0);
+                    tc_commit(empty + stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(tfull + acc);
+            }
+            if (!ok) gemm_signal_abort(args, abort_v);
+            // Every MMA this thread issued has completed before TMEM is released.
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0, nullptr, lim);
+        }
+    } else {
+        // ------------------------------------------------------- epilogue --
+        const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
+        const int r = quad * 32 + lane;
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(tfull + acc, acc_phase, abort_v, lim)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int n_blk = tile % args.num_n_tiles, m_blk = tile / args.num_n_tiles;
+
+            // Where this thread's accumulator row goes.
+            bool valid = true;
+            size_t dst_row = 0;  // element offset of column 0 of the row
+            int pos_row = 0;
+            if (args.conv) {
+                const int vr_local = r / args.conv_cols;
+                const int j = r - vr_local * args.conv_cols;
+                const int vr = m_blk * args.conv_rows + vr_local;
+                const int chunk = vr / args.conv_vrows;
+                const int i = vr - chunk * args.conv_vrows;
+                valid = vr_local < args.conv_rows && i < args.conv_vrows - 1 &&
+                        chunk < args.conv_chunks;
+                if (args.epi == kEpiConvPlanes) {
+                    // conv2 output (row i, col j) -> phase plane ((i&1), (j&1)) of conv3's input,
+                    // behind one zero row and one zero column.
+                    const int plane = (i & 1) * 2 + (j & 1);
+                    const size_t prow = (size_t)plane * args.dst_plane_rows +
+                                        (size_t)chunk * args.dst_chunk_rows + (i >> 1) + 1;
+                    dst_row = (prow * (size_t)args.dst_cols + (j >> 1) + 1) * (size_t)args.C;
+                } else {
+                    // conv3 output (mel row f = i, time j) -> token row chunk * 13 + j, column f*C.
+                    dst_row = ((size_t)(chunk * args.conv_cols + j) * (args.conv_vrows - 1) + i) *
+                              (size_t)args.C;
+                }
+            } else {
+                const int m = m_blk * 128 + r;
+                valid = m < args.M;
+                if (args.epi == kEpiPackTokens) {
+                    const int cl = m / kTokensPerChunkDev;
+                    const int t = m - cl * kTokensPerChunkDev;
+                    if (valid) {
+                        const int4 ci = args.chunks[args.chunk_base + cl];
+                        valid = t < stem_tokens_dev(ci.z);
+                        dst_row = (size_t)(ci.w + t) * args.ldo;
+                    }
+                    pos_row = t;
+                } else {
+                    dst_row = (size_t)m * args.ldo;
+                }
+            }
+
+            const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN / 16; ++c) {
+                float v[16];
+                tmem_ld16(t_addr + c * 16, v);
+                tc_wait_ld();
+                const int n0 = n_blk * BN + c * 16;
+                if (!valid) continue;
+                add_bias16(v, args.bias, n0);
+                switch (args.epi) {
+                    case kEpiBf16:
+                        store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
+                        break;
+                    case kEpiBf16Gelu:
+                    case kEpiConvPlanes:
+                    case kEpiConvFlat:
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = gelu_erf(v[i]);
+                        store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
+                        break;
+                    case kEpiResidF32:
+                    case kEpiPackTokens: {
+                        float4 *p = reinterpret_cast<float4 *>(reinterpret_cast<float *>(args.out) +
+                                                               dst_row + n0);
+                        if (args.epi == kEpiResidF32) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                float4 o = p[q];
+                                o.x += v[4 * q];
+                                o.y += v[4 * q + 1];
+                                o.z += v[4 * q + 2];
+                                o.w += v[4 * q + 3];
+                                p[q] = o;
+                            }
+                        } else {
+                            if (args.pos) {
+                                const float4 *pp = reinterpret_cast<const float4 *>(
+                                    args.pos + (size_t)pos_row * args.N + n0);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const float4 e = __ldg(pp + q);
+                                    v[4 * q] += e.x;
+                                    v[4 * q + 1] += e.y;
+                                    v[4 * q + 2] += e.z;
+                                    v[4 * q + 3] += e.w;
+                                }
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                                                   v[4 * q + 3]);
+                        }
+                        break;
+                    }
+                    default:
+                        break;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + acc);
+        }
+        if (!ok && lane == 0) gemm_signal_abort(args, abort_v);
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace aut

@@ -1,0 +1,470 @@
+// Non-GEMM kernels of the encoder: conv1 of the stem, LayerNorm, window
+// attention, one-time weight preparation, and small helpers.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "aut_internal.h"
+#include "aut_kernels.h"
+#include "aut_ptx.cuh"
+
+namespace aut {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ conv1 --
+// conv1 of the stem (aut_encoder page, module docstring; openarchlab "1A . AuT
+// Audio Encoder", section 3): Conv2d(1 -> C, k3, s2, p1) + GELU over one
+// 128 x 100 chunk whose frames at or after the request's length are zero (the
+// last chunk of a request is zero-padded to a full chunk, AuTEncoder.frontend).
+//
+// The 64 x 50 x C output goes to four phase planes P[(h&1)*2 + (w&1)], each
+// [33][26][C] per chunk with a zero row 0 and zero column 0 in front, holding
+// output (h, w) at (h/2 + 1, w/2 + 1).  conv2's filter tap (kh, kw) then reads
+// one plane at a fixed offset, a plain rectangle a TMA box can fetch.
+//
+// Block (chunk, 8 output rows); each thread computes channel pairs for a
+// strided set of positions, so a warp writes 32 consecutive channel pairs.
+__global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ feats, int T_max,
+                                                    const int4 *__restrict__ chunks,
+                                                    int chunk_base, const bf16 *__restrict__ w,
+                                                    const bf16 *__restrict__ b,
+                                                    bf16 *__restrict__ planes, int plane_rows,
+                                                    int C) {
+    const int cl = blockIdx.x, hg = blockIdx.y;
+    const int4 ci = chunks[chunk_base + cl];
+    __shared__ float xs[17][101];  // mel rows 16 hg - 1 .. 16 hg + 15, frames -1 .. 99
+    const bf16 *src = feats + ((size_t)ci.x * kMelBins) * T_max + ci.y;
+    for (int idx = threadIdx.x; idx < 17 * 101; idx += blockDim.x) {
+        const int rr = idx / 101, cc = idx - rr * 101;
+        const int mel = 16 * hg - 1 + rr, fr = cc - 1;
+        float v = 0.f;
+        if (mel >= 0 && mel < kMelBins && fr >= 0 && fr < ci.z)
+            v = __bfloat162float(src[(size_t)mel * T_max + fr]);
+        xs[rr][cc] = v;
+    }
+    __syncthreads();
+
+    const int CP = C >> 1;
+    const int slices = blockDim.x / CP;
+    const int cp = threadIdx.x % CP, slice = threadIdx.x / CP;
+    if (slice >= slices) return;
+    float w0[9], w1[9];
+#pragma unroll
+    for (int k = 0; k < 9; ++k) {
+        w0[k] = __bfloat162float(w[(2 * cp) * 9 + k]);
+        w1[k] = __bfloat162float(w[(2 * cp + 1) * 9 + k]);
+    }
+    const float b0 = __bfloat162float(b[2 * cp]), b1 = __bfloat162float(b[2 * cp + 1]);
+    const size_t chunk_row0 = (size_t)cl * kP1Rows;
+    for (int pos = slice; pos < 8 * kC1Cols; pos += slices) {
+        const int hl = pos / kC1Cols, wo = pos - hl * kC1Cols;
+        float a0 = b0, a1 = b1;
+#pragma unroll
+        for (int kh = 0; kh < 3; ++kh)
+#pragma unroll
+            for (int kw = 0; kw < 3; ++kw) {
+                const float x = xs[2 * hl + kh][2 * wo + kw];
+                a0 = fmaf(w0[kh * 3 + kw], x, a0);
+                a1 = fmaf(w1[kh * 3 + kw], x, a1);
+            }
+        const int h = 8 * hg + hl;
+        const int plane = (h & 1) * 2 + (wo & 1);
+        const size_t row = (size_t)plane * plane_rows + chunk_row0 + (h >> 1) + 1;
+        uint32_t *dst = reinterpret_cast<uint32_t *>(planes + (row * kP1Cols + (wo >> 1) + 1) * C) + cp;
+        *dst = pack_bf16x2(gelu_erf(a0), gelu_erf(a1));
+    }
+    // Zero column of the plane rows this block owns, and (first block) the zero row.
+    for (int idx = slice; idx < 16; idx += slices) {
+        const int plane = idx >> 2, r = 4 * hg + (idx & 3) + 1;
+        const size_t row = (size_t)plane * plane_rows + chunk_row0 + r;
+        reinterpret_cast<uint32_t *>(planes + row * kP1Cols * C)[cp] = 0u;
+    }
+    if (hg == 0)
+        for (int idx = slice; idx < 4 * kP1Cols; idx += slices) {
+            const int plane = idx / kP1Cols, col = idx - plane * kP1Cols;
+            const size_t row = (size_t)plane * plane_rows + chunk_row0;
+            reinterpret_cast<uint32_t *>(planes + (row * kP1Cols + col) * C)[cp] = 0u;
+        }
+}
+
+// Zero row, zero column and (odd-column planes) the missing last column of
+// conv3's input planes: the conv2 epilogue never writes them.
+__global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int plane_rows, int C) {
+    const int cl = blockIdx.x, plane = blockIdx.y;
+    const int CP = C >> 1;
+    const size_t row0 = (size_t)plane * plane_rows + (size_t)cl * kP2Rows;
+    const int extra = (plane & 1) ? (kP2Rows - 1) : 0;  // column kP2Cols - 1 of rows 1..16
+    const int n = (kP2Cols + (kP2Rows - 1) + extra) * CP;
+    for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
+        const int e = idx / CP, cp = idx - e * CP;
+        size_t row;
+        int col;
+        if (e < kP2Cols) {
+            row = row0;
+            col = e;
+        } else if (e < kP2Cols + kP2Rows - 1) {
+            row = row0 + 1 + (e - kP2Cols);
+            col = 0;
+        } else {
+            row = row0 + 1 + (e - kP2Cols - (kP2Rows - 1));
+            col = kP2Cols - 1;
+        }
+        reinterpret_cast<uint32_t *>(planes + (row * kP2Cols + col) * C)[cp] = 0u;
+    }
+}
+
+// -------------------------------------------------------------- layernorm --
+// LayerNorm with bias (cubic.dev "Audio Encoder Component", Transformer Encoder
+// Layers), fp32 in, bf16 out; one warp per row, the row held in registers,
+// two passes (mean, then centred variance).
+template <int VPL>  // float4 per lane
+__global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict__ x,
+                                                        const bf16 *__restrict__ g,
+                                                        const bf16 *__restrict__ bt,
+                                                        bf16 *__restrict__ y, int T, int d,
+                                                        float eps) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= T) return;
+    const int n4 = d >> 2;
+    const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)row * d);
+    float4 v[VPL];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int idx = lane + 32 * i;
+        if (idx < n4) {
+            v[i] = xr[idx];
+            s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / d;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int idx = lane + 32 * i;
+        if (idx < n4) {
+            const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, e = v[i].w - mean;
+            ss += (a * a + b * b) + (c * c + e * e);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rstd = rsqrtf(ss / d + eps);
+    uint2 *yr = reinterpret_cast<uint2 *>(y + (size_t)row * d);
+    const uint2 *gr = reinterpret_cast<const uint2 *>(g);
+    const uint2 *br = reinterpret_cast<const uint2 *>(bt);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int idx = lane + 32 * i;
+        if (idx < n4) {
+            const uint2 gg = __ldg(gr + idx), bb = __ldg(br + idx);
+            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg.x));
+            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg.y));
+            const float2 c0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb.x));
+            const float2 c1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb.y));
+            uint2 o;
+            o.x = pack_bf16x2((v[i].x - mean) * rstd * g0.x + c0.x, (v[i].y - mean) * rstd * g0.y + c0.y);
+            o.y = pack_bf16x2((v[i].z - mean) * rstd * g1.x + c1.x, (v[i].w - mean) * rstd * g1.y + c1.y);
+            yr[idx] = o;
+        }
+    }
+}
+
+// --------------------------------------------------------- window attention --
+AUT_DEV void ldmatrix_x4(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_addr(p)));
+}
+AUT_DEV void ldmatrix_x4_trans(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_addr(p)));
+}
+AUT_DEV void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Bidirectional attention inside one cu_seqlens window for one head (aut_encoder
+// page, AuTAttention: block-diagonal over the packed windows, no cache; openarchlab
+// "1A . AuT Audio Encoder", section 3: non-causal within each segment).  A window
+// has at most 128 tokens, so Q, K and V of one (window, head) sit in shared memory
+// whole and the softmax is exact in one pass: S = Q K^T (fp32), row max, exp,
+// row sum, O = P V / sum.  Keys past the window's length are masked; rows past it
+// are computed on zeros and not written.  Each warp owns 16-row query tiles.
+template <int HD>
+__global__ void __launch_bounds__(128) window_attn_kernel(const bf16 *__restrict__ qkv,
+                                                          bf16 *__restrict__ out,
+                                                          const int *__restrict__ cu, int d,
+                                                          float scale_log2e) {
+    constexpr int LD = HD + 8;  // padded row: conflict-free ldmatrix
+    extern __shared__ __align__(16) uint8_t attn_smem[];
+    bf16 *sQ = reinterpret_cast<bf16 *>(attn_smem);
+    bf16 *sK = sQ + kMaxWindowTokens * LD;
+    bf16 *sV = sK + kMaxWindowTokens * LD;
+    const int seg = blockIdx.x, h = blockIdx.y;
+    const int s0 = cu[seg], len = cu[seg + 1] - s0;
+    if (len <= 0) return;
+    const int nkt = (len + 15) >> 4;
+    const int rows = nkt * 16;
+    constexpr int CH = HD / 8;
+    for (int idx = threadIdx.x; idx < 3 * rows * CH; idx += blockDim.x) {
+        const int part = idx / (rows * CH);
+        const int rem = idx - part * rows * CH;
+        const int r = rem / CH, c = rem - (rem / CH) * CH;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (r < len)
+            val = __ldg(reinterpret_cast<const uint4 *>(qkv + (size_t)(s0 + r) * 3 * d + part * d +
+                                                        h * HD + c * 8));
+        bf16 *dst = (part == 0 ? sQ : part == 1 ? sK : sV) + r * LD + c * 8;
+        *reinterpret_cast<uint4 *>(dst) = val;
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    for (int mt = warp; mt < nkt; mt += 4) {
+        float s[16][4];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+            uint32_t a[4];
+            ldmatrix_x4(a, sQ + (mt * 16 + (lane & 15)) * LD + kk * 16 + (lane >> 4) * 8);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                if (nt < nkt) {
+                    uint32_t b[4];
+                    ldmatrix_x4(b, sK + (nt * 16 + (lane & 7) + ((lane >> 4) << 3)) * LD + kk * 16 +
+                                       ((lane >> 3) & 1) * 8);
+                    mma_16816(s[2 * nt], a, b[0], b[1]);
+                    mma_16816(s[2 * nt + 1], a, b[2], b[3]);
+                }
+            }
+        }
+        // exact softmax over the window's keys (rows g and g + 8 of the tile)
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (j < 2 * nkt) {
+                const int c0 = j * 8 + 2 * t;
+                if (c0 >= len) s[j][0] = s[j][2] = -INFINITY;
+                if (c0 + 1 >= len) s[j][1] = s[j][3] = -INFINITY;
+                mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
+                mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
+            }
+        }
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (j < 2 * nkt) {
+                s[j][0] = exp2f((s[j][0] - mx0) * scale_log2e);
+                s[j][1] = exp2f((s[j][1] - mx0) * scale_log2e);
+                s[j][2] = exp2f((s[j][2] - mx1) * scale_log2e);
+                s[j][3] = exp2f((s[j][3] - mx1) * scale_log2e);
+                sum0 += s[j][0] + s[j][1];
+                sum1 += s[j][2] + s[j][3];
+            }
+        }
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+            sum0 += __shfl_xor_sync(0xffffffffu, sum0, o);
+            sum1 += __shfl_xor_sync(0xffffffffu, sum1, o);
+        }
+        float o_acc[HD / 8][4];
+#pragma unroll
+        for (int j = 0; j < HD / 8; ++j) o_acc[j][0] = o_acc[j][1] = o_acc[j][2] = o_acc[j][3] = 0.f;
+#pragma unroll
+        for (int kt = 0; kt < 8; ++kt) {
+            if (kt < nkt) {
+                uint32_t pa[4];
+                pa[0] = pack_bf16x2(s[2 * kt][0], s[2 * kt][1]);
+                pa[1] = pack_bf16x2(s[2 * kt][2], s[2 * kt][3]);
+                pa[2] = pack_bf16x2(s[2 * kt + 1][0], s[2 * kt + 1][1]);
+                pa[3] = pack_bf16x2(s[2 * kt + 1][2], s[2 * kt + 1][3]);
+#pragma unroll
+                for (int np = 0; np < HD / 16; ++np) {
+                    uint32_t b[4];
+                    ldmatrix_x4_trans(b, sV + (kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LD +
+                                             np * 16 + (lane >> 4) * 8);
+                    mma_16816(o_acc[2 * np], pa, b[0], b[1]);
+                    mma_16816(o_acc[2 * np + 1], pa, b[2], b[3]);
+                }
+            }
+        }
+        const float inv0 = 1.f / sum0, inv1 = 1.f / sum1;
+        const int r0 = mt * 16 + g, r1 = r0 + 8;
+#pragma unroll
+        for (int j = 0; j < HD / 8; ++j) {
+            const int col = h * HD + j * 8 + 2 * t;
+            if (r0 < len)
+                *reinterpret_cast<uint32_t *>(out + (size_t)(s0 + r0) * d + col) =
+                    pack_bf16x2(o_acc[j][0] * inv0, o_acc[j][1] * inv0);
+            if (r1 < len)
+                *reinterpret_cast<uint32_t *>(out + (size_t)(s0 + r1) * d + col) =
+                    pack_bf16x2(o_acc[j][2] * inv1, o_acc[j][3] * inv1);
+        }
+    }
+}
+
+// -------------------------------------------------------------- prepare ----
+// conv weights [co][ci][kh][kw] -> [co][kh*3 + kw][ci] (channel-last per tap,
+// the "weight transposition" of the cubic.dev Audio Encoder page).
+__global__ void conv_tap_major_kernel(const bf16 *__restrict__ src, bf16 *__restrict__ dst, int C) {
+    const size_t n = (size_t)C * 9 * C;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const int ci = (int)(i % C);
+        const size_t rest = i / C;
+        const int tap = (int)(rest % 9);
+        const int co = (int)(rest / 9);
+        dst[i] = src[((size_t)co * C + ci) * 9 + tap];
+    }
+}
+
+// conv_out weight [d][c*16 + f] -> [d][f*C + c]: the stem writes its output
+// channel-fastest, so conv_out's K index is reordered once instead.
+__global__ void conv_out_reorder_kernel(const bf16 *__restrict__ src, bf16 *__restrict__ dst, int d,
+                                        int C) {
+    const size_t K = (size_t)kStemRows * C;
+    const size_t n = (size_t)d * K;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = i / K;
+        const int k = (int)(i - row * K);
+        const int f = k / C, c = k - f * C;
+        dst[i] = src[row * K + (size_t)c * kStemRows + f];
+    }
+}
+
+// Sinusoid table [13][d] (aut_encoder page, module docstring: the same 13
+// positions for every chunk; cubic.dev page: computed, never loaded), in the
+// Whisper form: row t = [sin(t g_k) | cos(t g_k)], g_k = exp(-k ln(1e4) / (d/2 - 1)),
+// evaluated in double and stored as fp32.
+__global__ void position_table_kernel(float *pos, int d) {
+    const int half = d / 2;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < kTokensPerChunk * d;
+         i += gridDim.x * blockDim.x) {
+        const int t = i / d, c = i - t * d;
+        const int k = c < half ? c : c - half;
+        const double inc = log(10000.0) / (double)(half - 1);
+        const double ang = (double)t * exp(-inc * (double)k);
+        pos[i] = (float)(c < half ? sin(ang) : cos(ang));
+    }
+}
+
+// Copies a block of 32-bit words carried in the kernel's parameters to device
+// memory: plan tables reach the device without a host buffer that has to
+// outlive the call.
+__global__ void upload_words_kernel(const UploadPayload p, int32_t *dst) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += gridDim.x * blockDim.x)
+        dst[p.offset + i] = p.words[i];
+}
+
+// ------------------------------------------------------------ launchers ----
+cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int chunk_base,
+                         int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
+                         int C, cudaStream_t st) {
+    if (n_chunks <= 0) return cudaSuccess;
+    conv1_kernel<<<dim3(n_chunks, kC1Rows / 8), 256, 0, st>>>(
+        static_cast<const bf16 *>(feats), T_max, chunks, chunk_base, static_cast<const bf16 *>(w),
+        static_cast<const bf16 *>(b), static_cast<bf16 *>(planes), plane_rows, C);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int C,
+                                   cudaStream_t st) {
+    if (n_chunks <= 0) return cudaSuccess;
+    zero_plane_pads_kernel<<<dim3(n_chunks, 4), 256, 0, st>>>(static_cast<bf16 *>(planes),
+                                                             plane_rows, C);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
+                             float eps, cudaStream_t st) {
+    if (T <= 0) return cudaSuccess;
+    const int vpl = (d / 4 + 31) / 32;
+    const dim3 grid((T + 7) / 8);
+    const bf16 *gg = static_cast<const bf16 *>(g), *bb = static_cast<const bf16 *>(b);
+    bf16 *yy = static_cast<bf16 *>(y);
+    if (vpl <= 4)
+        layernorm_kernel<4><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps);
+    else if (vpl <= 8)
+        layernorm_kernel<8><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps);
+    else
+        layernorm_kernel<16><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps);
+    return cudaGetLastError();
+}
+
+template <int HD>
+cudaError_t run_window_attention(const bf16 *q, bf16 *o, const int *cu_dev, int n_windows, int d,
+                                 int heads, float scale_log2e, cudaStream_t st) {
+    constexpr int smem = 3 * kMaxWindowTokens * (HD + 8) * (int)sizeof(bf16);
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(window_attn_kernel<HD>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
+    window_attn_kernel<HD><<<dim3(n_windows, heads), 128, smem, st>>>(q, o, cu_dev, d, scale_log2e);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
+                                    int d, int heads, cudaStream_t st) {
+    if (n_windows <= 0) return cudaSuccess;
+    const int hd = d / heads;
+    const float scale_log2e = 1.4426950408889634f / sqrtf((float)hd);
+    const bf16 *q = static_cast<const bf16 *>(qkv);
+    bf16 *o = static_cast<bf16 *>(out);
+    switch (hd) {
+        case 16: return run_window_attention<16>(q, o, cu_dev, n_windows, d, heads, scale_log2e, st);
+        case 32: return run_window_attention<32>(q, o, cu_dev, n_windows, d, heads, scale_log2e, st);
+        case 64: return run_window_attention<64>(q, o, cu_dev, n_windows, d, heads, scale_log2e, st);
+        case 128: return run_window_attention<128>(q, o, cu_dev, n_windows, d, heads, scale_log2e, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_prepare(const void *conv2_w, const void *conv3_w, const void *conv_out_w,
+                           void *conv2_tap, void *conv3_tap, void *conv_out_fc, float *pos, int C,
+                           int d, cudaStream_t st) {
+    conv_tap_major_kernel<<<592, 256, 0, st>>>(static_cast<const bf16 *>(conv2_w),
+                                               static_cast<bf16 *>(conv2_tap), C);
+    conv_tap_major_kernel<<<592, 256, 0, st>>>(static_cast<const bf16 *>(conv3_w),
+                                               static_cast<bf16 *>(conv3_tap), C);
+    conv_out_reorder_kernel<<<592, 256, 0, st>>>(static_cast<const bf16 *>(conv_out_w),
+                                                 static_cast<bf16 *>(conv_out_fc), d, C);
+    position_table_kernel<<<(kTokensPerChunk * d + 255) / 256, 256, 0, st>>>(pos, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_upload(const int32_t *host_words, size_t n, int32_t *dst, cudaStream_t st) {
+    UploadPayload p;
+    for (size_t off = 0; off < n; off += UploadPayload::kWords) {
+        p.n = (int)std::min<size_t>(UploadPayload::kWords, n - off);
+        p.offset = (int)off;
+        std::copy(host_words + off, host_words + off + p.n, p.words);
+        upload_words_kernel<<<(p.n + 255) / 256, 256, 0, st>>>(p, dst);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace aut

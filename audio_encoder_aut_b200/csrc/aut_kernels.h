@@ -1,0 +1,80 @@
+// Host launchers of the encoder's kernels (implemented in aut_kernels.cu and
+// aut_gemm.cu), used by the C-ABI layer in aut_api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace aut {
+
+enum GemmEpilogue : int {
+    kEpiBf16 = 0,        // out bf16 [M, ldo] = acc + bias
+    kEpiBf16Gelu = 1,    // out bf16 [M, ldo] = GELU(acc + bias)
+    kEpiResidF32 = 2,    // out fp32 [M, ldo] += acc + bias
+    kEpiConvPlanes = 3,  // conv2: GELU(acc + bias) -> conv3's phase planes
+    kEpiConvFlat = 4,    // conv3: GELU(acc + bias) -> [chunk * 13 + t][f * C + c]
+    kEpiPackTokens = 5,  // conv_out: acc (+ bias) (+ pos[t]) -> packed fp32 rows
+};
+
+struct UploadPayload {
+    static constexpr int kWords = 8000;  // 32,000 bytes: within the kernel-parameter limit
+    int n, offset;
+    int32_t words[kWords];
+};
+
+cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int chunk_base,
+                         int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
+                         int C, cudaStream_t st);
+cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int C,
+                                   cudaStream_t st);
+cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
+                             float eps, cudaStream_t st);
+cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
+                                    int d, int heads, cudaStream_t st);
+cudaError_t launch_prepare(const void *conv2_w, const void *conv3_w, const void *conv_out_w,
+                           void *conv2_tap, void *conv3_tap, void *conv_out_fc, float *pos, int C,
+                           int d, cudaStream_t st);
+cudaError_t launch_upload(const int32_t *host_words, size_t n, int32_t *dst, cudaStream_t st);
+
+// ---- tensor-core GEMMs (aut_gemm.cu) ----
+enum class GemmStatus { kOk, kBadShape, kTensorMap, kLaunch };
+
+struct LinearLaunch {
+    const void *a;     // bf16 [M, K]
+    const void *w;     // bf16 [N, K]
+    const void *bias;  // bf16 [N] or null
+    void *out;
+    int M, N, K, ldo;
+    int epi;           // GemmEpilogue
+    // pack-tokens epilogue
+    const int4 *chunks;
+    int chunk_base;
+    const float *pos;
+    int *status;
+    unsigned long long timeout_ns;
+    int fault_inject;
+};
+GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st);
+
+struct ConvLaunch {
+    const void *planes;  // bf16 [4][plane_rows_cap][cols_in][C]: input phase planes
+    int plane_rows_cap;  // rows of one plane in the buffer
+    int chunks;          // chunks in this group
+    int chunk_rows;      // plane rows per chunk (33 for conv2, 17 for conv3), zero row included
+    int cols_in;         // plane columns, zero column included (26 / 14)
+    int out_cols;        // output columns (25 / 13)
+    int rows_per_tile;   // virtual rows per 128-row M tile (5 / 9)
+    int C;
+    const void *w_tap;   // bf16 [C][9][C]
+    const void *bias;    // bf16 [C]
+    int epi;             // kEpiConvPlanes (conv2) or kEpiConvFlat (conv3)
+    void *out;
+    int dst_plane_rows, dst_chunk_rows, dst_cols;  // kEpiConvPlanes destination geometry
+    int *status;
+    unsigned long long timeout_ns;
+};
+GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st);
+
+}  // namespace aut

@@ -1,0 +1,130 @@
+"""PyTorch plumbing around the C ABI: device buffers for the weights, the
+workspace and the outputs, and the current CUDA stream.  Nothing here computes
+any step of the encoder; every step runs in libaut.so."""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _lib as A
+
+
+def _dev_bf16(arr, device) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32))
+    return t.to(device=device, dtype=torch.bfloat16).contiguous()
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def current_stream_handle(device=None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+class Encoder:
+    """Holds one encoder's weights on a GPU and runs it through libaut.so.
+
+    `cfg` has AuTEncoderConfig-style attributes; `weights` is a dict of arrays
+    in PyTorch layouts (see include/aut.h), e.g. from aut_synth.weights()."""
+
+    def __init__(self, cfg, weights: dict, device: int | str = 0):
+        if not torch.cuda.is_available():
+            raise RuntimeError("the AuT encoder runs on a CUDA GPU only")
+        self.device = torch.device("cuda", torch.device(device).index
+                                   if isinstance(device, str) else device)
+        self.cfg = cfg
+        self.c = A.make_config(cfg)
+        A.lib()
+        dev = self.device
+        self._keep = []
+
+        def up(a):
+            if a is None:
+                return None
+            t = _dev_bf16(a, dev)
+            self._keep.append(t)
+            return t
+
+        w = A.aut_weights()
+        for k in ["conv1_w", "conv1_b", "conv2_w", "conv2_b", "conv3_w", "conv3_b",
+                  "conv_out_w", "conv_out_b", "ln_post_w", "ln_post_b", "proj1_w", "proj1_b",
+                  "proj2_w", "proj2_b"]:
+            setattr(w, k, _ptr(up(weights.get(k))))
+        n = len(weights["layers"])
+        self._layers = (A.aut_layer_weights * max(1, n))()
+        for i, lw in enumerate(weights["layers"]):
+            for k in A.LAYER_FIELDS:
+                setattr(self._layers[i], k, _ptr(up(lw[k])))
+        w.layers = ctypes.cast(self._layers, ctypes.POINTER(A.aut_layer_weights))
+        self._src = w
+        nbytes = A.aut_prepared_bytes(self.c)
+        if nbytes == 0:
+            raise A.AutError(A.AUT_ERR_UNSUPPORTED, "aut_prepared_bytes")
+        self._prepared_buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        with torch.cuda.device(dev):
+            self.prepared = A.aut_prepare_weights(self.c, self._src, self._prepared_buf.data_ptr(),
+                                                  nbytes, current_stream_handle(dev))
+        self._ws = None
+
+    # ------------------------------------------------------------------
+    def plan(self, feature_lens):
+        return A.aut_plan(self.c, feature_lens)
+
+    def workspace(self, total_tokens: int, num_windows: int, num_chunks: int) -> torch.Tensor:
+        need = A.aut_workspace_bytes(self.c, total_tokens, num_windows, num_chunks)
+        if need == 0:
+            raise A.AutError(A.AUT_ERR_UNSUPPORTED, "aut_workspace_bytes")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def features_to_device(self, feats: np.ndarray) -> torch.Tensor:
+        return _dev_bf16(feats, self.device)
+
+    def encode(self, features: torch.Tensor, feature_lens, out: torch.Tensor | None = None):
+        """features: bf16 [B, 128, T_max] on the device -> bf16 [total_tokens, output_dim]."""
+        _, _, total, nw, nch = self.plan(feature_lens)
+        ws = self.workspace(total, nw, nch)
+        if out is None:
+            out = torch.empty((total, self.cfg.output_dim), dtype=torch.bfloat16, device=self.device)
+        st = A.aut_encode(self.c, self.prepared, features.data_ptr(), features.shape[-1],
+                          feature_lens, out.data_ptr(), ws.data_ptr(), ws.numel(),
+                          current_stream_handle(self.device))
+        if st != A.AUT_OK:
+            raise A.AutError(st, "aut_encode")
+        return out
+
+    def frontend(self, features: torch.Tensor, feature_lens, with_positions: bool = True):
+        """-> fp32 [total_tokens, d_model] packed chunk embeddings."""
+        _, _, total, nw, nch = self.plan(feature_lens)
+        ws = self.workspace(total, nw, nch)
+        x0 = torch.empty((total, self.cfg.d_model), dtype=torch.float32, device=self.device)
+        st = A.aut_frontend(self.c, self.prepared, features.data_ptr(), features.shape[-1],
+                            feature_lens, x0.data_ptr(), with_positions, ws.data_ptr(), ws.numel(),
+                            current_stream_handle(self.device))
+        if st != A.AUT_OK:
+            raise A.AutError(st, "aut_frontend")
+        return x0
+
+    def encode_packed(self, hidden: torch.Tensor, cu_seqlens, n_layers: int,
+                      with_projector: bool = True):
+        """Runs layers [0, n_layers) on `hidden` (fp32 [T, d], updated in place) and
+        optionally the projector; returns the projector output or None."""
+        T = hidden.shape[0]
+        ws = self.workspace(T, len(cu_seqlens) - 1, 0)
+        out = None
+        if with_projector:
+            out = torch.empty((T, self.cfg.output_dim), dtype=torch.bfloat16, device=self.device)
+        st = A.aut_encode_packed(self.c, self.prepared, hidden.data_ptr(), T, cu_seqlens, n_layers,
+                                 _ptr(out), ws.data_ptr(), ws.numel(),
+                                 current_stream_handle(self.device))
+        if st != A.AUT_OK:
+            raise A.AutError(st, "aut_encode_packed")
+        return out
+
+    def check(self) -> int:
+        """Device status of the latest call on this encoder's workspace."""
+        return A.aut_check(self._ws.data_ptr()) if self._ws is not None else A.AUT_OK

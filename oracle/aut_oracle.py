@@ -224,22 +224,30 @@ def stem(cfg, w: dict, mel: np.ndarray, dtype=np.float64) -> np.ndarray:
 
 
 def frontend(cfg, w: dict, feats: np.ndarray, feature_lens, dtype=np.float64,
-             with_positions: bool = True, chunk_batch: int = 16) -> np.ndarray:
+             with_positions: bool = True, chunk_batch: int = 16,
+             stem_rows: dict | None = None) -> np.ndarray:
     """(B, mel, T_max) zero-padded mel + valid lengths -> packed
     [total_tokens, d_model] [aut_encoder, AuTEncoder.frontend]: every chunk gets
     the same tokens_per_chunk positions, then is trimmed to its valid tokens and
-    packed chunk by chunk, request by request."""
+    packed chunk by chunk, request by request.  If `stem_rows` is a dict, the
+    packed rows before the positions are added are also stored under "stem"."""
     layout = plan(cfg, feature_lens)
     tpc = tokens_per_chunk(cfg)
     pe = sinusoids(tpc, cfg.d_model, dtype)
     x0 = np.zeros((layout.total_tokens, cfg.d_model), dtype=dtype)
+    raw = np.zeros_like(x0) if stem_rows is not None else None
     for s in range(0, len(layout.chunks), chunk_batch):
         part = layout.chunks[s:s + chunk_batch]
         h = stem(cfg, w, chunk_mel(cfg, feats, layout, part, dtype), dtype)
+        if raw is not None:
+            for c, hc in zip(part, h):
+                raw[c.token0:c.token0 + c.valid_tokens] = hc[:c.valid_tokens]
         if with_positions:
             h = h + pe[None]
         for c, hc in zip(part, h):
             x0[c.token0:c.token0 + c.valid_tokens] = hc[:c.valid_tokens]
+    if stem_rows is not None:
+        stem_rows["stem"] = raw
     return x0
 
 
@@ -311,9 +319,11 @@ def encode(cfg, w: dict, x0: np.ndarray, cu_seqlens, hidden: dict | None = None)
 def forward(cfg, w: dict, feats: np.ndarray, feature_lens, dtype=np.float64,
             hidden: dict | None = None):
     """features, feature_lens -> (out [total_tokens, output_dim], layout)
-    [aut_encoder, AuTEncoder.forward]."""
+    [aut_encoder, AuTEncoder.forward].  If `hidden` is a dict it receives the
+    stem rows before positions ("stem"), x0 ("x0") and the residual stream
+    after every layer (layer index)."""
     layout = plan(cfg, feature_lens)
-    x0 = frontend(cfg, w, feats, feature_lens, dtype)
+    x0 = frontend(cfg, w, feats, feature_lens, dtype, stem_rows=hidden)
     if hidden is not None:
         hidden["x0"] = x0
     return encode(cfg, w, x0, layout.cu_seqlens, hidden), layout

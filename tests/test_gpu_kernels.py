@@ -1,0 +1,144 @@
+"""Kernel-level parity on the GPU, through the C ABI: the tcgen05 linear layer
+and its epilogues, LayerNorm and window attention against the oracle's
+definitions on the same bf16 inputs; the bounded-wait timeout status."""
+import numpy as np
+import pytest
+
+import aut_synth as S
+import oracle as O
+from gpu_util import assert_rows_close
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from audio_encoder_aut_b200 import _lib as A  # noqa: E402
+
+
+def _dev(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda").to(dtype)
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _rand(shape, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return S.round_bf16(rng.standard_normal(shape).astype(np.float32) * scale)
+
+
+SHAPES = [(1, 64, 64), (31, 192, 64), (128, 256, 256), (300, 1280, 1280), (1000, 3840, 1280),
+          (257, 2688, 896), (390, 3584, 896), (77, 16, 64), (129, 240, 7680), (4000, 5120, 1280),
+          (3000, 1280, 5120), (513, 2048, 1280), (45, 1024, 896)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("epi", [A.EPI_BF16, A.EPI_BF16_GELU, A.EPI_RESID_F32])
+def test_linear_matches_definition(M, N, K, epi):
+    x = _rand((M, K), 1)
+    w = _rand((N, K), 2, 0.05)
+    b = _rand((N,), 3, 0.1)
+    ref = x.astype(np.float64) @ w.astype(np.float64).T + b
+    xd, wd, bd = _dev(x, torch.bfloat16), _dev(w, torch.bfloat16), _dev(b, torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if epi == A.EPI_RESID_F32:
+        y0 = np.random.default_rng(4).standard_normal((M, N)).astype(np.float32)
+        yd = _dev(y0, torch.float32)
+        ref = ref + y0
+    else:
+        yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        if epi == A.EPI_BF16_GELU:
+            ref = O.gelu(ref)
+    st = A.aut_linear(xd.data_ptr(), wd.data_ptr(), bd.data_ptr(), yd.data_ptr(), M, N, K, epi,
+                      status.data_ptr(), 0, 0, _stream())
+    assert st == A.AUT_OK
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = yd.float().cpu().numpy()
+    if epi == A.EPI_RESID_F32:
+        # fp32 output: only accumulation-order error
+        np.testing.assert_allclose(got, ref, rtol=0, atol=2e-3 * np.sqrt(K / 64))
+    else:
+        assert_rows_close(got, ref, f"linear {M}x{N}x{K} epi {epi}")
+
+
+def test_linear_no_bias_and_structured_inputs():
+    """Identity-like A picks out rows of W: checks operand layout and K order exactly."""
+    M, N, K = 128, 256, 256
+    x = np.zeros((M, K), np.float32)
+    for i in range(M):
+        x[i, (3 * i) % K] = 1.0
+    w = _rand((N, K), 5)
+    yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    st = A.aut_linear(_dev(x, torch.bfloat16).data_ptr(), _dev(w, torch.bfloat16).data_ptr(),
+                      None, yd.data_ptr(), M, N, K, A.EPI_BF16, None, 0, 0, _stream())
+    assert st == A.AUT_OK
+    torch.cuda.synchronize()
+    ref = np.stack([w[:, (3 * i) % K] for i in range(M)])
+    np.testing.assert_array_equal(yd.float().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("T,d", [(1, 64), (31, 64), (390, 896), (3200, 1280), (17, 2048)])
+def test_layernorm_matches_oracle(T, d):
+    rng = np.random.default_rng(T)
+    x = (rng.standard_normal((T, d)) * 2 + 0.5).astype(np.float32)
+    g = S.round_bf16(1 + 0.1 * rng.standard_normal(d).astype(np.float32))
+    b = S.round_bf16(0.1 * rng.standard_normal(d).astype(np.float32))
+    y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    st = A.aut_layernorm(_dev(x, torch.float32).data_ptr(), _dev(g, torch.bfloat16).data_ptr(),
+                         _dev(b, torch.bfloat16).data_ptr(), y.data_ptr(), T, d, 1e-5, _stream())
+    assert st == A.AUT_OK
+    torch.cuda.synchronize()
+    ref = O.layer_norm(x.astype(np.float64), g, b, 1e-5)
+    assert_rows_close(y.float().cpu().numpy(), ref, "layernorm")
+    np.testing.assert_allclose(y.float().cpu().numpy(), ref, rtol=1e-2, atol=1e-2)
+
+
+ATTN_CASES = [
+    (4, 16, [26, 5]),
+    (20, 64, [104, 104, 1, 17, 128, 50, 104, 3]),
+    (14, 64, [104, 104, 104, 78]),
+    (2, 32, [7, 64, 33]),
+    (2, 128, [100, 1, 128]),
+]
+
+
+@pytest.mark.parametrize("heads,hd,lens", ATTN_CASES)
+def test_window_attention_matches_oracle(heads, hd, lens):
+    d = heads * hd
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    T = cu[-1]
+    qkv = _rand((T, 3 * d), 11, 1.0)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    st = A.aut_window_attention(_dev(qkv, torch.bfloat16).data_ptr(), out.data_ptr(), T, d, heads,
+                                cu, ws.data_ptr(), ws.numel(), _stream())
+    assert st == A.AUT_OK
+    torch.cuda.synchronize()
+    ref = O.window_attention(qkv.astype(np.float64), cu, heads)
+    assert_rows_close(out.float().cpu().numpy(), ref, "window attention")
+
+
+def test_pipeline_wait_timeout_returns_status_and_gpu_stays_usable():
+    """A GEMM whose first block never receives its first operand tile: the
+    consumer's bounded wait runs out, the kernel records AUT_ERR_TIMEOUT and
+    returns; the next launch on the same context works."""
+    M, N, K = 256, 128, 128
+    x = _dev(_rand((M, K), 1), torch.bfloat16)
+    w = _dev(_rand((N, K), 2, 0.05), torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = A.aut_linear(x.data_ptr(), w.data_ptr(), None, y.data_ptr(), M, N, K, A.EPI_BF16,
+                      status.data_ptr(), 200, 1, _stream())
+    assert st == A.AUT_OK
+    torch.cuda.synchronize()
+    assert A.aut_check_status_word(status.data_ptr()) == A.AUT_ERR_TIMEOUT
+    assert int(status.item()) == 0  # cleared by the check
+    st = A.aut_linear(x.data_ptr(), w.data_ptr(), None, y.data_ptr(), M, N, K, A.EPI_BF16,
+                      status.data_ptr(), 0, 0, _stream())
+    torch.cuda.synchronize()
+    assert st == A.AUT_OK and A.aut_check_status_word(status.data_ptr()) == A.AUT_OK
+    ref = x.float().cpu().numpy().astype(np.float64) @ w.float().cpu().numpy().astype(np.float64).T
+    assert_rows_close(y.float().cpu().numpy(), ref, "linear after timeout")
