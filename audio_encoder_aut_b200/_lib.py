@@ -15,7 +15,11 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 AUT_OK, AUT_ERR_INVALID_ARG, AUT_ERR_UNSUPPORTED, AUT_ERR_WORKSPACE, AUT_ERR_CUDA, \
     AUT_ERR_TIMEOUT = range(6)
 
-EPI_BF16, EPI_BF16_GELU, EPI_RESID_F32 = 0, 1, 2
+EPI_BF16, EPI_BF16_GELU, EPI_RESID_F32, EPI_F32 = 0, 1, 2, 3
+
+KERNEL_KINDS = ["upload", "zero_pads", "conv1", "conv2", "conv3", "conv_out", "layernorm",
+                "qkv", "attention", "o_proj", "fc1", "fc2", "proj1", "proj2"]
+GEMM_KINDS = {"conv2", "conv3", "conv_out", "qkv", "o_proj", "fc1", "fc2", "proj1", "proj2"}
 
 
 class aut_config(ctypes.Structure):
@@ -39,7 +43,13 @@ class aut_weights(ctypes.Structure):
                 + [("layers", POINTER(aut_layer_weights))]
                 + [(n, c_void_p) for n in ["ln_post_w", "ln_post_b", "proj1_w", "proj1_b",
                                            "proj2_w", "proj2_b", "conv2_w_tap", "conv3_w_tap",
-                                           "conv_out_w_fc", "pos_table"]])
+                                           "conv_out_w_fc", "pos_table", "proj1_w_dup",
+                                           "proj2_w_dup", "o_w_dup"]])
+
+
+class aut_trace(ctypes.Structure):
+    _fields_ = [("events", POINTER(c_void_p)), ("capacity", c_int32), ("count", c_int32),
+                ("kinds", POINTER(c_int32))]
 
 
 class AutError(RuntimeError):
@@ -60,6 +70,9 @@ _SIGNATURES = {
                                       c_size_t, POINTER(aut_weights), c_void_p]),
     "aut_encode": (c_int32, [POINTER(aut_config), POINTER(aut_weights), c_void_p, c_int32,
                              POINTER(c_int32), c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "aut_encode_traced": (c_int32, [POINTER(aut_config), POINTER(aut_weights), c_void_p, c_int32,
+                                    POINTER(c_int32), c_int32, c_void_p, c_void_p, c_size_t,
+                                    c_void_p, POINTER(aut_trace)]),
     "aut_frontend": (c_int32, [POINTER(aut_config), POINTER(aut_weights), c_void_p, c_int32,
                                POINTER(c_int32), c_int32, c_void_p, c_int32, c_void_p, c_size_t,
                                c_void_p]),
@@ -170,6 +183,13 @@ def aut_encode(cfg, prepared, features: int, t_max: int, feature_lens, out: int,
     return lib().aut_encode(ctypes.byref(cfg), ctypes.byref(prepared), features, t_max,
                             _i32(feature_lens), len(feature_lens), out, workspace, ws_bytes,
                             stream)
+
+
+def aut_encode_traced(cfg, prepared, features: int, t_max: int, feature_lens, out: int,
+                      workspace: int, ws_bytes: int, stream: int, trace: aut_trace | None) -> int:
+    return lib().aut_encode_traced(ctypes.byref(cfg), ctypes.byref(prepared), features, t_max,
+                                   _i32(feature_lens), len(feature_lens), out, workspace, ws_bytes,
+                                   stream, ctypes.byref(trace) if trace is not None else None)
 
 
 def aut_frontend(cfg, prepared, features: int, t_max: int, feature_lens, x0: int,

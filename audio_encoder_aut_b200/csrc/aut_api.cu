@@ -36,7 +36,7 @@ struct Region {
 };
 
 struct PreparedLayout {
-    size_t conv2, conv3, conv_out, pos, total;
+    size_t conv2, conv3, conv_out, pos, proj1_dup, proj2_dup, o_dup, total;
 };
 
 PreparedLayout prepared_layout(const aut_config *c) {
@@ -47,6 +47,9 @@ PreparedLayout prepared_layout(const aut_config *c) {
     p.conv3 = r.take(C * 9 * C * 2);
     p.conv_out = r.take(d * kStemRows * C * 2);
     p.pos = r.take((size_t)kTokensPerChunk * d * 4);
+    p.proj1_dup = r.take(d * 2 * d * 2);
+    p.proj2_dup = r.take((size_t)c->output_dim * 2 * d * 2);
+    p.o_dup = r.take((size_t)std::max(c->layers, 1) * d * 2 * d * 2);
     p.total = r.off;
     return p;
 }
@@ -73,15 +76,15 @@ bool weights_complete(const aut_config *c, const aut_weights *w, int n_layers, b
     if (stem && (!w->conv1_w || !w->conv1_b || !w->conv2_b || !w->conv3_b || !w->conv2_w_tap ||
                  !w->conv3_w_tap || !w->conv_out_w_fc || !w->pos_table))
         return false;
-    if (n_layers > 0 && !w->layers) return false;
+    if (n_layers > 0 && (!w->layers || !w->o_w_dup)) return false;
     for (int i = 0; i < n_layers; ++i) {
         const aut_layer_weights &l = w->layers[i];
         if (!l.ln1_w || !l.ln1_b || !l.qkv_w || !l.qkv_b || !l.o_w || !l.o_b || !l.ln2_w ||
             !l.ln2_b || !l.fc1_w || !l.fc1_b || !l.fc2_w || !l.fc2_b)
             return false;
     }
-    if (projector && (!w->ln_post_w || !w->ln_post_b || !w->proj1_w || !w->proj1_b ||
-                      !w->proj2_w || !w->proj2_b))
+    if (projector && (!w->ln_post_w || !w->ln_post_b || !w->proj1_b || !w->proj2_b ||
+                      !w->proj1_w_dup || !w->proj2_w_dup))
         return false;
     (void)c;
     return true;
@@ -94,6 +97,20 @@ struct Ctx {
     WorkspaceLayout L;
     cudaStream_t st;
     int *status;
+    aut_trace *trace = nullptr;
+
+    // Records the trace event after a kernel launch (no-op without a trace).
+    aut_status mark(int kind) const {
+        if (!trace) return AUT_OK;
+        const int i = trace->count++;
+        if (i < trace->capacity) {
+            if (trace->kinds) trace->kinds[i] = kind;
+            if (trace->events &&
+                cudaEventRecord(static_cast<cudaEvent_t>(trace->events[i]), st) != cudaSuccess)
+                return AUT_ERR_CUDA;
+        }
+        return AUT_OK;
+    }
 
     template <class T>
     T *at(size_t off) const {
@@ -102,7 +119,7 @@ struct Ctx {
 };
 
 aut_status linear(const Ctx &c, const void *a, const void *w, const void *b, void *out, int M,
-                  int N, int K, int epi) {
+                  int N, int K, int epi, int kind, int ldo = 0) {
     LinearLaunch L{};
     L.a = a;
     L.w = w;
@@ -111,11 +128,12 @@ aut_status linear(const Ctx &c, const void *a, const void *w, const void *b, voi
     L.M = M;
     L.N = N;
     L.K = K;
-    L.ldo = N;
+    L.ldo = ldo ? ldo : N;
     L.epi = epi;
     L.status = c.status;
     L.timeout_ns = kDefaultTimeoutNs;
-    return gemm_status(launch_linear(L, c.st));
+    AUT_TRY(gemm_status(launch_linear(L, c.st)));
+    return c.mark(kind);
 }
 
 aut_status upload_plan(const Ctx &c, const Plan &p) {
@@ -128,8 +146,10 @@ aut_status upload_plan(const Ctx &c, const Plan &p) {
         words.push_back(ci.token0);
     }
     AUT_TRY(cuda_status(launch_upload(words.data(), words.size(), c.at<int32_t>(c.L.chunks), c.st)));
-    return cuda_status(
-        launch_upload(p.cu_seqlens.data(), p.cu_seqlens.size(), c.at<int32_t>(c.L.cu), c.st));
+    AUT_TRY(c.mark(AUT_K_UPLOAD));
+    AUT_TRY(cuda_status(
+        launch_upload(p.cu_seqlens.data(), p.cu_seqlens.size(), c.at<int32_t>(c.L.cu), c.st)));
+    return c.mark(AUT_K_UPLOAD);
 }
 
 // AuTEncoder.frontend: chunks -> conv stem -> conv_out + positions -> packed x0.
@@ -146,10 +166,12 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
     void *y3 = c.at<void>(c.L.y3);
     const int p1_rows = G * kP1Rows, p2_rows = G * kP2Rows;
     AUT_TRY(cuda_status(launch_zero_plane_pads(planes2, p2_rows, G, C, c.st)));
+    AUT_TRY(c.mark(AUT_K_ZERO_PADS));
     for (int c0 = 0; c0 < n_ch; c0 += G) {
         const int g = std::min(G, n_ch - c0);
         AUT_TRY(cuda_status(launch_conv1(feats, T_max, chunks, c0, g, c.w->conv1_w, c.w->conv1_b,
                                          planes1, p1_rows, C, c.st)));
+        AUT_TRY(c.mark(AUT_K_CONV1));
         ConvLaunch k2{};
         k2.planes = planes1;
         k2.plane_rows_cap = p1_rows;
@@ -169,6 +191,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
         k2.status = c.status;
         k2.timeout_ns = kDefaultTimeoutNs;
         AUT_TRY(gemm_status(launch_conv_gemm(k2, c.st)));
+        AUT_TRY(c.mark(AUT_K_CONV2));
         ConvLaunch k3 = k2;
         k3.planes = planes2;
         k3.plane_rows_cap = p2_rows;
@@ -181,6 +204,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
         k3.epi = kEpiConvFlat;
         k3.out = y3;
         AUT_TRY(gemm_status(launch_conv_gemm(k3, c.st)));
+        AUT_TRY(c.mark(AUT_K_CONV3));
         LinearLaunch lo{};
         lo.a = y3;
         lo.w = c.w->conv_out_w_fc;
@@ -197,6 +221,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
         lo.status = c.status;
         lo.timeout_ns = kDefaultTimeoutNs;
         AUT_TRY(gemm_status(launch_linear(lo, c.st)));
+        AUT_TRY(c.mark(AUT_K_CONV_OUT));
     }
     return AUT_OK;
 }
@@ -213,23 +238,39 @@ aut_status run_encode(const Ctx &c, float *x, int T, int nW, int n_layers, void 
     for (int l = 0; l < n_layers; ++l) {
         const aut_layer_weights &lw = c.w->layers[l];
         AUT_TRY(cuda_status(launch_layernorm(x, lw.ln1_w, lw.ln1_b, xn, T, d, cfg->ln_eps, c.st)));
-        AUT_TRY(linear(c, xn, lw.qkv_w, lw.qkv_b, qkv, T, 3 * d, d, kEpiBf16));
+        AUT_TRY(c.mark(AUT_K_LAYERNORM));
+        AUT_TRY(linear(c, xn, lw.qkv_w, lw.qkv_b, qkv, T, 3 * d, d, kEpiBf16, AUT_K_QKV));
         AUT_TRY(cuda_status(launch_window_attention(qkv, attn, cu, nW, d, cfg->heads, c.st)));
-        AUT_TRY(linear(c, attn, lw.o_w, lw.o_b, x, T, d, d, kEpiResidF32));
+        AUT_TRY(c.mark(AUT_K_ATTENTION));
+        // attention output [hi | lo] against [o_w | o_w]
+        const void *o_w2 = static_cast<const uint8_t *>(c.w->o_w_dup) + (size_t)l * d * 2 * d * 2;
+        AUT_TRY(linear(c, attn, o_w2, lw.o_b, x, T, d, 2 * d, kEpiResidF32, AUT_K_O_PROJ));
         AUT_TRY(cuda_status(launch_layernorm(x, lw.ln2_w, lw.ln2_b, xn, T, d, cfg->ln_eps, c.st)));
-        AUT_TRY(linear(c, xn, lw.fc1_w, lw.fc1_b, ffn, T, F, d, kEpiBf16Gelu));
-        AUT_TRY(linear(c, ffn, lw.fc2_w, lw.fc2_b, x, T, d, F, kEpiResidF32));
+        AUT_TRY(c.mark(AUT_K_LAYERNORM));
+        AUT_TRY(linear(c, xn, lw.fc1_w, lw.fc1_b, ffn, T, F, d, kEpiBf16Gelu, AUT_K_FC1));
+        AUT_TRY(linear(c, ffn, lw.fc2_w, lw.fc2_b, x, T, d, F, kEpiResidF32, AUT_K_FC2));
     }
     if (!out) return AUT_OK;
+    // Projector operands as hi + lo bf16 pairs ([hi | lo] rows against K-repeated
+    // weights): its two roundings would otherwise add as much error as a layer.
     AUT_TRY(cuda_status(
-        launch_layernorm(x, c.w->ln_post_w, c.w->ln_post_b, xn, T, d, cfg->ln_eps, c.st)));
-    AUT_TRY(linear(c, xn, c.w->proj1_w, c.w->proj1_b, ffn, T, d, d, kEpiBf16Gelu));
-    return linear(c, ffn, c.w->proj2_w, c.w->proj2_b, out, T, cfg->output_dim, d, kEpiBf16);
+        launch_layernorm(x, c.w->ln_post_w, c.w->ln_post_b, xn, T, d, cfg->ln_eps, c.st, true)));
+    AUT_TRY(c.mark(AUT_K_LAYERNORM));
+    AUT_TRY(linear(c, xn, c.w->proj1_w_dup, c.w->proj1_b, ffn, T, d, 2 * d, kEpiBf16GeluSplit,
+                   AUT_K_PROJ1, 2 * d));
+    return linear(c, ffn, c.w->proj2_w_dup, c.w->proj2_b, out, T, cfg->output_dim, 2 * d,
+                  kEpiF32, AUT_K_PROJ2);
 }
 
 aut_status make_ctx(const aut_config *cfg, const aut_weights *w, void *ws, size_t ws_bytes,
-                    const Plan &p, cudaStream_t st, Ctx *c) {
+                    const Plan &p, cudaStream_t st, Ctx *c, aut_trace *trace = nullptr) {
     c->cfg = cfg;
+    c->trace = trace;
+    if (trace) {
+        if (trace->capacity < 0 || (trace->capacity > 0 && !trace->events && !trace->kinds))
+            return AUT_ERR_INVALID_ARG;
+        trace->count = 0;
+    }
     c->w = w;
     c->ws = static_cast<uint8_t *>(ws);
     c->st = st;
@@ -262,10 +303,10 @@ WorkspaceLayout workspace_layout(const aut_config *c, int64_t T, int64_t nW, int
     // The stem buffers and the layer buffers are never live together: overlay them.
     const size_t base = r.off;
     Region a{base};
-    L.xn = a.take((size_t)T * d * 2);
+    L.xn = a.take((size_t)T * 2 * d * 2);  // [hi | lo] rows for the projector
     L.qkv = a.take((size_t)T * 3 * d * 2);
-    L.attn = a.take((size_t)T * d * 2);
-    L.ffn = a.take((size_t)T * std::max(F, d) * 2);
+    L.attn = a.take((size_t)T * 2 * d * 2);  // [hi | lo] rows
+    L.ffn = a.take((size_t)T * std::max(F, 2 * d) * 2);
     const int G = (int)std::min<int64_t>(n_ch, c->conv_chunksize);
     L.group_chunks = G;
     Region b{base};
@@ -296,7 +337,8 @@ extern "C" aut_status aut_prepare_weights(const aut_config *cfg, const aut_weigh
                                           size_t dst_bytes, aut_weights *prepared,
                                           aut_stream_t stream) {
     AUT_TRY(check_config(cfg));
-    if (!src || !dst || !prepared || !src->conv2_w || !src->conv3_w || !src->conv_out_w)
+    if (!src || !dst || !prepared || !src->conv2_w || !src->conv3_w || !src->conv_out_w ||
+        !src->proj1_w || !src->proj2_w)
         return AUT_ERR_INVALID_ARG;
     const PreparedLayout p = prepared_layout(cfg);
     if (dst_bytes < p.total) return AUT_ERR_WORKSPACE;
@@ -307,6 +349,21 @@ extern "C" aut_status aut_prepare_weights(const aut_config *cfg, const aut_weigh
     out.conv3_w_tap = base + p.conv3;
     out.conv_out_w_fc = base + p.conv_out;
     out.pos_table = base + p.pos;
+    out.proj1_w_dup = base + p.proj1_dup;
+    out.proj2_w_dup = base + p.proj2_dup;
+    out.o_w_dup = base + p.o_dup;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (int l = 0; l < cfg->layers; ++l) {
+        if (!src->layers || !src->layers[l].o_w) return AUT_ERR_INVALID_ARG;
+        AUT_TRY(cuda_status(launch_duplicate_k(src->layers[l].o_w,
+                                               base + p.o_dup + (size_t)l * cfg->d_model * 2 *
+                                                                    cfg->d_model * 2,
+                                               cfg->d_model, cfg->d_model, st)));
+    }
+    AUT_TRY(cuda_status(launch_duplicate_k(src->proj1_w, base + p.proj1_dup, cfg->d_model,
+                                           cfg->d_model, st)));
+    AUT_TRY(cuda_status(launch_duplicate_k(src->proj2_w, base + p.proj2_dup, cfg->output_dim,
+                                           cfg->d_model, st)));
     AUT_TRY(cuda_status(launch_prepare(src->conv2_w, src->conv3_w, src->conv_out_w,
                                        base + p.conv2, base + p.conv3, base + p.conv_out,
                                        reinterpret_cast<float *>(base + p.pos), cfg->conv_ch,
@@ -319,13 +376,24 @@ extern "C" aut_status aut_encode(const aut_config *cfg, const aut_weights *prepa
                                  const void *features, int32_t T_max, const int32_t *feature_lens,
                                  int32_t n_req, void *out, void *workspace, size_t ws_bytes,
                                  aut_stream_t stream) {
+    return aut_encode_traced(cfg, prepared, features, T_max, feature_lens, n_req, out, workspace,
+                             ws_bytes, stream, nullptr);
+}
+
+extern "C" aut_status aut_encode_traced(const aut_config *cfg, const aut_weights *prepared,
+                                        const void *features, int32_t T_max,
+                                        const int32_t *feature_lens, int32_t n_req, void *out,
+                                        void *workspace, size_t ws_bytes, aut_stream_t stream,
+                                        aut_trace *trace) {
     Plan p;
     AUT_TRY(build_plan(cfg, feature_lens, n_req, &p));
     AUT_TRY(check_features(p, features, T_max, feature_lens, n_req));
     if (!weights_complete(cfg, prepared, cfg->layers, true, true)) return AUT_ERR_INVALID_ARG;
     if (p.total_tokens > 0 && !out) return AUT_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(out) & 15u) return AUT_ERR_INVALID_ARG;
     Ctx c;
-    AUT_TRY(make_ctx(cfg, prepared, workspace, ws_bytes, p, reinterpret_cast<cudaStream_t>(stream), &c));
+    AUT_TRY(make_ctx(cfg, prepared, workspace, ws_bytes, p, reinterpret_cast<cudaStream_t>(stream),
+                     &c, trace));
     if (p.total_tokens == 0) return AUT_OK;
     AUT_TRY(upload_plan(c, p));
     float *x = c.at<float>(c.L.x);
@@ -382,7 +450,7 @@ extern "C" aut_status aut_encode_packed(const aut_config *cfg, const aut_weights
 extern "C" aut_status aut_linear(const void *x, const void *w, const void *bias, void *y, int32_t M,
                                  int32_t N, int32_t K, int32_t epilogue, int32_t *status,
                                  int32_t timeout_ms, int32_t fault_inject, aut_stream_t stream) {
-    if (M < 0 || N <= 0 || K <= 0 || epilogue < 0 || epilogue > 2 || timeout_ms < 0)
+    if (M < 0 || N <= 0 || K <= 0 || epilogue < 0 || epilogue > 3 || timeout_ms < 0)
         return AUT_ERR_INVALID_ARG;
     if (M > 0 && (!x || !w || !y)) return AUT_ERR_INVALID_ARG;
     if (K % 64 || N % 16) return AUT_ERR_UNSUPPORTED;
@@ -395,7 +463,7 @@ extern "C" aut_status aut_linear(const void *x, const void *w, const void *bias,
     L.N = N;
     L.K = K;
     L.ldo = N;
-    L.epi = epilogue;
+    L.epi = epilogue == 3 ? kEpiF32 : epilogue;
     L.status = reinterpret_cast<int *>(status);
     L.timeout_ns = timeout_ms ? (unsigned long long)timeout_ms * 1000000ull : kDefaultTimeoutNs;
     L.fault_inject = fault_inject ? 1 : 0;

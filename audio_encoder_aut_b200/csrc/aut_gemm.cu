@@ -69,7 +69,7 @@ GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &arg
     }
     const int tiles = args.num_m_tiles * args.num_n_tiles;
     const int grid = std::min(tiles, sm_count());
-    gemm_tc_kernel<BN><<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, args);
+    gemm_tc_kernel<BN><<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, args);
     return cudaGetLastError() == cudaSuccess ? GemmStatus::kOk : GemmStatus::kLaunch;
 }
 

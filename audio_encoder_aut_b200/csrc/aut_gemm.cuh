@@ -11,10 +11,10 @@
 //     past the chunk's valid length and writes each kept row to its packed
 //     position (token packing fused into the GEMM).
 //
-// Block = 6 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory
+// Block = 10 warps: warp 0 issues TMA loads into a STAGES-deep shared-memory
 // ring, warp 1 owns the tensor-memory allocation and issues tcgen05.mma from
-// one thread, warps 2-5 drain the accumulator (tcgen05.ld) and run the
-// epilogue.  Two accumulators in tensor memory let the epilogue of one tile
+// one thread, warps 2-9 drain the accumulator (tcgen05.ld) and run the
+// epilogue (two warps per 32-lane TMEM quadrant).  Two accumulators in tensor memory let the epilogue of one tile
 // overlap the MMAs of the next.  Tiles are 128 x BN x 64 (bf16, 128-byte
 // swizzle); the grid is persistent (one CTA per SM, tiles strided by gridDim).
 // Every mbarrier wait is bounded: on time-out the kernel records
@@ -28,6 +28,8 @@
 namespace aut {
 
 constexpr int kTokensPerChunkDev = 13;  // tokens out of one 100-frame chunk
+constexpr int kEpilogueWarps = 8;
+constexpr int kGemmThreads = 64 + 32 * kEpilogueWarps;  // producer warp, MMA warp, epilogue
 
 // Epilogue codes (GemmEpilogue) are declared in aut_kernels.h.
 
@@ -122,7 +124,7 @@ AUT_DEV void add_bias16(float (&v)[16], const __nv_bfloat16 *bias, int n0) {
 }
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs args) {
     using Cfg = GemmCfg<BN>;
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, 4);
+            mbar_init(tempty + a, kEpilogueWarps);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -265,8 +267,13 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         // ------------------------------------------------------- epilogue --
+        // Eight warps: TMEM lane quadrant (warp % 4) x column half (alternate
+        // 16-column chunks).  Two chunks are loaded per TMEM wait, and the
+        // residual rows they update are fetched before that wait.
         const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
+        const int half = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
+        constexpr int NC = BN / 16;
         int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
@@ -322,40 +329,65 @@ __global__ void __launch_bounds__(192, 1)
 
             const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
-            for (int c = 0; c < BN / 16; ++c) {
-                float v[16];
-                tmem_ld16(t_addr + c * 16, v);
+            for (int c0 = half; c0 < NC; c0 += 4) {
+                const int c1 = c0 + 2;
+                const bool two = c1 < NC;  // warp-uniform
+                float v0[16], v1[16];
+                tmem_ld16(t_addr + c0 * 16, v0);
+                if (two) tmem_ld16(t_addr + c1 * 16, v1);
+                float4 res0[4], res1[4];
+                float *rp = reinterpret_cast<float *>(args.out) + dst_row;
+                if (args.epi == kEpiResidF32 && valid) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) res0[q] = reinterpret_cast<const float4 *>(rp + c0 * 16 + n_blk * BN)[q];
+                    if (two)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) res1[q] = reinterpret_cast<const float4 *>(rp + c1 * 16 + n_blk * BN)[q];
+                }
                 tc_wait_ld();
-                const int n0 = n_blk * BN + c * 16;
                 if (!valid) continue;
-                add_bias16(v, args.bias, n0);
-                switch (args.epi) {
-                    case kEpiBf16:
-                        store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
-                        break;
-                    case kEpiBf16Gelu:
-                    case kEpiConvPlanes:
-                    case kEpiConvFlat:
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = gelu_erf(v[i]);
-                        store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
-                        break;
-                    case kEpiResidF32:
-                    case kEpiPackTokens: {
-                        float4 *p = reinterpret_cast<float4 *>(reinterpret_cast<float *>(args.out) +
-                                                               dst_row + n0);
-                        if (args.epi == kEpiResidF32) {
+                for (int k = 0; k < 2; ++k) {
+                    if (k == 1 && !two) break;
+                    float(&v)[16] = k ? v1 : v0;
+                    const float4(&res)[4] = k ? res1 : res0;
+                    const int n0 = n_blk * BN + (k ? c1 : c0) * 16;
+                    add_bias16(v, args.bias, n0);
+                    switch (args.epi) {
+                        case kEpiBf16:
+                            store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
+                            break;
+                        case kEpiBf16Gelu:
+                        case kEpiConvPlanes:
+                        case kEpiConvFlat:
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                float4 o = p[q];
-                                o.x += v[4 * q];
-                                o.y += v[4 * q + 1];
-                                o.z += v[4 * q + 2];
-                                o.w += v[4 * q + 3];
-                                p[q] = o;
+                            for (int i = 0; i < 16; ++i) v[i] = gelu_fast(v[i]);
+                            store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
+                            break;
+                        case kEpiBf16GeluSplit: {
+                            // GELU, then the value as hi + lo bf16 halves [hi | lo] of a 2N row.
+                            float lo[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                v[i] = gelu_fast(v[i]);
+                                lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
                             }
-                        } else {
-                            if (args.pos) {
+                            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0;
+                            store_bf16x16(o, v);
+                            store_bf16x16(o + args.N, lo);
+                            break;
+                        }
+                        case kEpiResidF32: {
+                            float4 *p = reinterpret_cast<float4 *>(rp + n0);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                p[q] = make_float4(res[q].x + v[4 * q], res[q].y + v[4 * q + 1],
+                                                   res[q].z + v[4 * q + 2], res[q].w + v[4 * q + 3]);
+                            break;
+                        }
+                        case kEpiF32:
+                        case kEpiPackTokens: {
+                            if (args.epi == kEpiPackTokens && args.pos) {
                                 const float4 *pp = reinterpret_cast<const float4 *>(
                                     args.pos + (size_t)pos_row * args.N + n0);
 #pragma unroll
@@ -367,15 +399,15 @@ __global__ void __launch_bounds__(192, 1)
                                     v[4 * q + 3] += e.w;
                                 }
                             }
+                            float4 *p = reinterpret_cast<float4 *>(rp + n0);
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
-                                p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
-                                                   v[4 * q + 3]);
+                                p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                            break;
                         }
-                        break;
+                        default:
+                            break;
                     }
-                    default:
-                        break;
                 }
             }
             tc_fence_before();

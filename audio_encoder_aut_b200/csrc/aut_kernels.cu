@@ -22,8 +22,8 @@ using bf16 = __nv_bfloat16;
 // output (h, w) at (h/2 + 1, w/2 + 1).  conv2's filter tap (kh, kw) then reads
 // one plane at a fixed offset, a plain rectangle a TMA box can fetch.
 //
-// Block (chunk, 8 output rows); each thread computes channel pairs for a
-// strided set of positions, so a warp writes 32 consecutive channel pairs.
+// Block (chunk, 8 output rows); each thread computes four channels for a
+// strided set of positions, so a warp writes 32 consecutive channel quads.
 __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ feats, int T_max,
                                                     const int4 *__restrict__ chunks,
                                                     int chunk_base, const bf16 *__restrict__ w,
@@ -44,46 +44,50 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
     }
     __syncthreads();
 
-    const int CP = C >> 1;
-    const int slices = blockDim.x / CP;
-    const int cp = threadIdx.x % CP, slice = threadIdx.x / CP;
+    const int CQ = C >> 2;  // channel quads
+    const int slices = blockDim.x / CQ;
+    const int cq = threadIdx.x % CQ, slice = threadIdx.x / CQ;
     if (slice >= slices) return;
-    float w0[9], w1[9];
+    float wt[4][9], bias[4];
 #pragma unroll
-    for (int k = 0; k < 9; ++k) {
-        w0[k] = __bfloat162float(w[(2 * cp) * 9 + k]);
-        w1[k] = __bfloat162float(w[(2 * cp + 1) * 9 + k]);
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int k = 0; k < 9; ++k) wt[c][k] = __bfloat162float(w[(4 * cq + c) * 9 + k]);
+        bias[c] = __bfloat162float(b[4 * cq + c]);
     }
-    const float b0 = __bfloat162float(b[2 * cp]), b1 = __bfloat162float(b[2 * cp + 1]);
     const size_t chunk_row0 = (size_t)cl * kP1Rows;
     for (int pos = slice; pos < 8 * kC1Cols; pos += slices) {
         const int hl = pos / kC1Cols, wo = pos - hl * kC1Cols;
-        float a0 = b0, a1 = b1;
+        float x[9];
 #pragma unroll
         for (int kh = 0; kh < 3; ++kh)
 #pragma unroll
-            for (int kw = 0; kw < 3; ++kw) {
-                const float x = xs[2 * hl + kh][2 * wo + kw];
-                a0 = fmaf(w0[kh * 3 + kw], x, a0);
-                a1 = fmaf(w1[kh * 3 + kw], x, a1);
-            }
+            for (int kw = 0; kw < 3; ++kw) x[kh * 3 + kw] = xs[2 * hl + kh][2 * wo + kw];
+        float a[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            a[c] = bias[c];
+#pragma unroll
+            for (int k = 0; k < 9; ++k) a[c] = fmaf(wt[c][k], x[k], a[c]);
+        }
         const int h = 8 * hg + hl;
         const int plane = (h & 1) * 2 + (wo & 1);
         const size_t row = (size_t)plane * plane_rows + chunk_row0 + (h >> 1) + 1;
-        uint32_t *dst = reinterpret_cast<uint32_t *>(planes + (row * kP1Cols + (wo >> 1) + 1) * C) + cp;
-        *dst = pack_bf16x2(gelu_erf(a0), gelu_erf(a1));
+        uint2 *dst = reinterpret_cast<uint2 *>(planes + (row * kP1Cols + (wo >> 1) + 1) * C) + cq;
+        *dst = make_uint2(pack_bf16x2(gelu_fast(a[0]), gelu_fast(a[1])),
+                          pack_bf16x2(gelu_fast(a[2]), gelu_fast(a[3])));
     }
     // Zero column of the plane rows this block owns, and (first block) the zero row.
     for (int idx = slice; idx < 16; idx += slices) {
         const int plane = idx >> 2, r = 4 * hg + (idx & 3) + 1;
         const size_t row = (size_t)plane * plane_rows + chunk_row0 + r;
-        reinterpret_cast<uint32_t *>(planes + row * kP1Cols * C)[cp] = 0u;
+        reinterpret_cast<uint2 *>(planes + row * kP1Cols * C)[cq] = make_uint2(0u, 0u);
     }
     if (hg == 0)
         for (int idx = slice; idx < 4 * kP1Cols; idx += slices) {
             const int plane = idx / kP1Cols, col = idx - plane * kP1Cols;
             const size_t row = (size_t)plane * plane_rows + chunk_row0;
-            reinterpret_cast<uint32_t *>(planes + (row * kP1Cols + col) * C)[cp] = 0u;
+            reinterpret_cast<uint2 *>(planes + (row * kP1Cols + col) * C)[cq] = make_uint2(0u, 0u);
         }
 }
 
@@ -116,18 +120,31 @@ __global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int 
 // -------------------------------------------------------------- layernorm --
 // LayerNorm with bias (cubic.dev "Audio Encoder Component", Transformer Encoder
 // Layers), fp32 in, bf16 out; one warp per row, the row held in registers,
-// two passes (mean, then centred variance).
+// two passes (mean, then centred variance).  With `split`, the output row is
+// [hi | lo] (2 d wide): hi = bf16(y), lo = bf16(y - hi), so that a GEMM over
+// the doubled K against [W | W] sees y to about 16 significant bits.
 template <int VPL>  // float4 per lane
 __global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict__ x,
                                                         const bf16 *__restrict__ g,
                                                         const bf16 *__restrict__ bt,
                                                         bf16 *__restrict__ y, int T, int d,
-                                                        float eps) {
+                                                        float eps, int split) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * 8 + warp;
     if (row >= T) return;
     const int n4 = d >> 2;
     const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)row * d);
+    const uint2 *gr = reinterpret_cast<const uint2 *>(g);
+    const uint2 *br = reinterpret_cast<const uint2 *>(bt);
+    uint2 gg[VPL], bb[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {  // gamma/beta in flight while the row is reduced
+        const int idx = lane + 32 * i;
+        if (idx < n4) {
+            gg[i] = __ldg(gr + idx);
+            bb[i] = __ldg(br + idx);
+        }
+    }
     float4 v[VPL];
     float s = 0.f;
 #pragma unroll
@@ -153,22 +170,30 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict_
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rstd = rsqrtf(ss / d + eps);
-    uint2 *yr = reinterpret_cast<uint2 *>(y + (size_t)row * d);
-    const uint2 *gr = reinterpret_cast<const uint2 *>(g);
-    const uint2 *br = reinterpret_cast<const uint2 *>(bt);
+    uint2 *yr = reinterpret_cast<uint2 *>(y + (size_t)row * (split ? 2 * d : d));
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
         const int idx = lane + 32 * i;
         if (idx < n4) {
-            const uint2 gg = __ldg(gr + idx), bb = __ldg(br + idx);
-            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg.x));
-            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg.y));
-            const float2 c0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb.x));
-            const float2 c1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb.y));
+            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg[i].x));
+            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg[i].y));
+            const float2 c0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb[i].x));
+            const float2 c1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb[i].y));
+            const float o0 = (v[i].x - mean) * rstd * g0.x + c0.x;
+            const float o1 = (v[i].y - mean) * rstd * g0.y + c0.y;
+            const float o2 = (v[i].z - mean) * rstd * g1.x + c1.x;
+            const float o3 = (v[i].w - mean) * rstd * g1.y + c1.y;
             uint2 o;
-            o.x = pack_bf16x2((v[i].x - mean) * rstd * g0.x + c0.x, (v[i].y - mean) * rstd * g0.y + c0.y);
-            o.y = pack_bf16x2((v[i].z - mean) * rstd * g1.x + c1.x, (v[i].w - mean) * rstd * g1.y + c1.y);
+            o.x = pack_bf16x2(o0, o1);
+            o.y = pack_bf16x2(o2, o3);
             yr[idx] = o;
+            if (split) {  // second half of the row: what bf16 rounding left out
+                const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162 *>(&o.x);
+                const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162 *>(&o.y);
+                const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+                yr[n4 + idx] = make_uint2(pack_bf16x2(o0 - f0.x, o1 - f0.y),
+                                          pack_bf16x2(o2 - f1.x, o3 - f1.y));
+            }
         }
     }
 }
@@ -198,9 +223,13 @@ AUT_DEV void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint3
 // has at most 128 tokens, so Q, K and V of one (window, head) sit in shared memory
 // whole and the softmax is exact in one pass: S = Q K^T (fp32), row max, exp,
 // row sum, O = P V / sum.  Keys past the window's length are masked; rows past it
-// are computed on zeros and not written.  Each warp owns 16-row query tiles.
+// are computed on zeros and not written.  Each of the 8 warps owns 16-row query
+// tiles.  P and the output carry a second bf16 term (hi + lo): the o_proj GEMM
+// that consumes the output then sees it to about 16 significant bits.
+constexpr int kAttnWarps = 8;
+
 template <int HD>
-__global__ void __launch_bounds__(128) window_attn_kernel(const bf16 *__restrict__ qkv,
+__global__ void __launch_bounds__(32 * kAttnWarps) window_attn_kernel(const bf16 *__restrict__ qkv,
                                                           bf16 *__restrict__ out,
                                                           const int *__restrict__ cu, int d,
                                                           float scale_log2e) {
@@ -215,22 +244,24 @@ __global__ void __launch_bounds__(128) window_attn_kernel(const bf16 *__restrict
     const int nkt = (len + 15) >> 4;
     const int rows = nkt * 16;
     constexpr int CH = HD / 8;
+    // Asynchronous 16-byte copies straight into shared memory, all in flight at
+    // once; rows past the window's end are zero-filled (source size 0).
     for (int idx = threadIdx.x; idx < 3 * rows * CH; idx += blockDim.x) {
         const int part = idx / (rows * CH);
         const int rem = idx - part * rows * CH;
         const int r = rem / CH, c = rem - (rem / CH) * CH;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (r < len)
-            val = __ldg(reinterpret_cast<const uint4 *>(qkv + (size_t)(s0 + r) * 3 * d + part * d +
-                                                        h * HD + c * 8));
+        const bf16 *src = qkv + (size_t)(s0 + (r < len ? r : 0)) * 3 * d + part * d + h * HD + c * 8;
         bf16 *dst = (part == 0 ? sQ : part == 1 ? sK : sV) + r * LD + c * 8;
-        *reinterpret_cast<uint4 *>(dst) = val;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
+                     "l"(src), "r"(r < len ? 16 : 0)
+                     : "memory");
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    for (int mt = warp; mt < nkt; mt += 4) {
+    for (int mt = warp; mt < nkt; mt += kAttnWarps) {
         float s[16][4];
 #pragma unroll
         for (int j = 0; j < 16; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
@@ -289,32 +320,50 @@ __global__ void __launch_bounds__(128) window_attn_kernel(const bf16 *__restrict
 #pragma unroll
         for (int kt = 0; kt < 8; ++kt) {
             if (kt < nkt) {
-                uint32_t pa[4];
-                pa[0] = pack_bf16x2(s[2 * kt][0], s[2 * kt][1]);
-                pa[1] = pack_bf16x2(s[2 * kt][2], s[2 * kt][3]);
-                pa[2] = pack_bf16x2(s[2 * kt + 1][0], s[2 * kt + 1][1]);
-                pa[3] = pack_bf16x2(s[2 * kt + 1][2], s[2 * kt + 1][3]);
+                // P as hi + lo bf16 terms: two MMAs against the same V fragment.
+                uint32_t ph[4], pl[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float(&sa)[4] = s[2 * kt + (q >> 1)];
+                    const float a = sa[(q & 1) * 2], b = sa[(q & 1) * 2 + 1];
+                    ph[q] = pack_bf16x2(a, b);
+                    const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ph[q]));
+                    pl[q] = pack_bf16x2(a - hf.x, b - hf.y);
+                }
 #pragma unroll
                 for (int np = 0; np < HD / 16; ++np) {
                     uint32_t b[4];
                     ldmatrix_x4_trans(b, sV + (kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LD +
                                              np * 16 + (lane >> 4) * 8);
-                    mma_16816(o_acc[2 * np], pa, b[0], b[1]);
-                    mma_16816(o_acc[2 * np + 1], pa, b[2], b[3]);
+                    mma_16816(o_acc[2 * np], ph, b[0], b[1]);
+                    mma_16816(o_acc[2 * np + 1], ph, b[2], b[3]);
+                    mma_16816(o_acc[2 * np], pl, b[0], b[1]);
+                    mma_16816(o_acc[2 * np + 1], pl, b[2], b[3]);
                 }
             }
         }
+        // O / rowsum written as [hi | lo] bf16 halves of a 2 d row.
         const float inv0 = 1.f / sum0, inv1 = 1.f / sum1;
         const int r0 = mt * 16 + g, r1 = r0 + 8;
 #pragma unroll
         for (int j = 0; j < HD / 8; ++j) {
             const int col = h * HD + j * 8 + 2 * t;
-            if (r0 < len)
-                *reinterpret_cast<uint32_t *>(out + (size_t)(s0 + r0) * d + col) =
-                    pack_bf16x2(o_acc[j][0] * inv0, o_acc[j][1] * inv0);
-            if (r1 < len)
-                *reinterpret_cast<uint32_t *>(out + (size_t)(s0 + r1) * d + col) =
-                    pack_bf16x2(o_acc[j][2] * inv1, o_acc[j][3] * inv1);
+            if (r0 < len) {
+                const float a = o_acc[j][0] * inv0, b = o_acc[j][1] * inv0;
+                const uint32_t hi = pack_bf16x2(a, b);
+                const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hi));
+                bf16 *o = out + (size_t)(s0 + r0) * 2 * d + col;
+                *reinterpret_cast<uint32_t *>(o) = hi;
+                *reinterpret_cast<uint32_t *>(o + d) = pack_bf16x2(a - hf.x, b - hf.y);
+            }
+            if (r1 < len) {
+                const float a = o_acc[j][2] * inv1, b = o_acc[j][3] * inv1;
+                const uint32_t hi = pack_bf16x2(a, b);
+                const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hi));
+                bf16 *o = out + (size_t)(s0 + r1) * 2 * d + col;
+                *reinterpret_cast<uint32_t *>(o) = hi;
+                *reinterpret_cast<uint32_t *>(o + d) = pack_bf16x2(a - hf.x, b - hf.y);
+            }
         }
     }
 }
@@ -393,18 +442,18 @@ cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, i
 }
 
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
-                             float eps, cudaStream_t st) {
+                             float eps, cudaStream_t st, bool split) {
     if (T <= 0) return cudaSuccess;
     const int vpl = (d / 4 + 31) / 32;
     const dim3 grid((T + 7) / 8);
     const bf16 *gg = static_cast<const bf16 *>(g), *bb = static_cast<const bf16 *>(b);
     bf16 *yy = static_cast<bf16 *>(y);
     if (vpl <= 4)
-        layernorm_kernel<4><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps);
+        layernorm_kernel<4><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps, split);
     else if (vpl <= 8)
-        layernorm_kernel<8><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps);
+        layernorm_kernel<8><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps, split);
     else
-        layernorm_kernel<16><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps);
+        layernorm_kernel<16><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps, split);
     return cudaGetLastError();
 }
 
@@ -421,7 +470,8 @@ cudaError_t run_window_attention(const bf16 *q, bf16 *o, const int *cu_dev, int 
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    window_attn_kernel<HD><<<dim3(n_windows, heads), 128, smem, st>>>(q, o, cu_dev, d, scale_log2e);
+    window_attn_kernel<HD><<<dim3(n_windows, heads), 32 * kAttnWarps, smem, st>>>(q, o, cu_dev, d,
+                                                                                  scale_log2e);
     return cudaGetLastError();
 }
 
@@ -439,6 +489,25 @@ cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_de
         case 128: return run_window_attention<128>(q, o, cu_dev, n_windows, d, heads, scale_log2e, st);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// [W | W]: a weight repeated along K, so that one GEMM over a [hi | lo] operand
+// accumulates W hi + W lo.
+__global__ void duplicate_k_kernel(const bf16 *__restrict__ src, bf16 *__restrict__ dst, int N,
+                                   int K) {
+    const size_t n = (size_t)N * 2 * K;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = i / (2 * K);
+        const int k = (int)(i - row * 2 * K);
+        dst[i] = src[row * K + (k < K ? k : k - K)];
+    }
+}
+
+cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st) {
+    duplicate_k_kernel<<<592, 256, 0, st>>>(static_cast<const bf16 *>(src), static_cast<bf16 *>(dst),
+                                            N, K);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_prepare(const void *conv2_w, const void *conv3_w, const void *conv_out_w,

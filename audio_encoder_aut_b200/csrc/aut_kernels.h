@@ -16,6 +16,8 @@ enum GemmEpilogue : int {
     kEpiConvPlanes = 3,  // conv2: GELU(acc + bias) -> conv3's phase planes
     kEpiConvFlat = 4,    // conv3: GELU(acc + bias) -> [chunk * 13 + t][f * C + c]
     kEpiPackTokens = 5,  // conv_out: acc (+ bias) (+ pos[t]) -> packed fp32 rows
+    kEpiF32 = 6,         // out fp32 [M, ldo] = acc + bias
+    kEpiBf16GeluSplit = 7,  // out bf16 [M, 2N]: GELU(acc + bias) as hi | lo halves
 };
 
 struct UploadPayload {
@@ -30,7 +32,8 @@ cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int c
 cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int C,
                                    cudaStream_t st);
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
-                             float eps, cudaStream_t st);
+                             float eps, cudaStream_t st, bool split = false);
+cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st);
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                     int d, int heads, cudaStream_t st);
 cudaError_t launch_prepare(const void *conv2_w, const void *conv3_w, const void *conv_out_w,

@@ -171,7 +171,21 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            ((uint32_t)(M >> 4) << 24);
 }
 
-AUT_DEV float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+// GELU(x) = x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2 (the exact form), with erf
+// from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z),
+// z >= 0, |error| <= 1.5e-7; odd symmetry for z < 0.
+AUT_DEV float gelu_fast(float x) {
+    const float z = fabsf(x) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+    float p = fmaf(1.061405429f, t, -1.453152027f);
+    p = fmaf(p, t, 1.421413741f);
+    p = fmaf(p, t, -0.284496736f);
+    p = fmaf(p, t, 0.254829592f);
+    p *= t;
+    const float erf_abs = fmaf(-p, __expf(-z * z), 1.0f);
+    return 0.5f * x * (1.0f + copysignf(erf_abs, x));
+}
 
 AUT_DEV uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);

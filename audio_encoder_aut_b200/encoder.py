@@ -84,15 +84,16 @@ class Encoder:
     def features_to_device(self, feats: np.ndarray) -> torch.Tensor:
         return _dev_bf16(feats, self.device)
 
-    def encode(self, features: torch.Tensor, feature_lens, out: torch.Tensor | None = None):
-        """features: bf16 [B, 128, T_max] on the device -> bf16 [total_tokens, output_dim]."""
+    def encode(self, features: torch.Tensor, feature_lens, out: torch.Tensor | None = None,
+               trace: A.aut_trace | None = None):
+        """features: bf16 [B, 128, T_max] on the device -> fp32 [total_tokens, output_dim]."""
         _, _, total, nw, nch = self.plan(feature_lens)
         ws = self.workspace(total, nw, nch)
         if out is None:
-            out = torch.empty((total, self.cfg.output_dim), dtype=torch.bfloat16, device=self.device)
-        st = A.aut_encode(self.c, self.prepared, features.data_ptr(), features.shape[-1],
-                          feature_lens, out.data_ptr(), ws.data_ptr(), ws.numel(),
-                          current_stream_handle(self.device))
+            out = torch.empty((total, self.cfg.output_dim), dtype=torch.float32, device=self.device)
+        st = A.aut_encode_traced(self.c, self.prepared, features.data_ptr(), features.shape[-1],
+                                 feature_lens, out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                 current_stream_handle(self.device), trace)
         if st != A.AUT_OK:
             raise A.AutError(st, "aut_encode")
         return out
@@ -117,7 +118,7 @@ class Encoder:
         ws = self.workspace(T, len(cu_seqlens) - 1, 0)
         out = None
         if with_projector:
-            out = torch.empty((T, self.cfg.output_dim), dtype=torch.bfloat16, device=self.device)
+            out = torch.empty((T, self.cfg.output_dim), dtype=torch.float32, device=self.device)
         st = A.aut_encode_packed(self.c, self.prepared, hidden.data_ptr(), T, cu_seqlens, n_layers,
                                  _ptr(out), ws.data_ptr(), ws.numel(),
                                  current_stream_handle(self.device))

@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Throughput of the AuT audio-encoder forward on B200 (one process per GPU).
+
+One step = one full forward (plan upload, conv stem, 24 pre-LN layers with
+window attention, final LN and projector) over one batch of synthetic log-mel
+input resident in HBM.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload omni_16req]
+  python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on
+the launching stream, with a 256 MiB buffer written between steps (L2 flush,
+outside the events); barrier + synchronize around the timed region; the
+device time is the max over ranks.  Weak scaling: every rank encodes its own
+batch of the same shape (different features, same weights); no collective is
+on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import aut_synth as S  # noqa: E402
+
+METRIC = "encoded audio-seconds/s on 1 B200 (bf16); tokens/s and % of bf16 TC peak alongside"
+UNIT = "audio-s/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["bf16_tflops"], d["bf16_tflops_sustained"], d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------ FLOP credit ----
+def _half(n):
+    return (n + 1) // 2 if n > 0 else 0
+
+
+def credited_flops(cfg, lens, cu):
+    """Algorithmic FLOPs of one forward, valid positions only: the stem per chunk
+    (conv1, conv2, conv3 on the output positions the chunk's valid frames reach,
+    conv_out on its kept tokens), 2 (4 d^2 + 2 d F) per token and layer for the
+    layer GEMMs, 4 d len^2 per window and layer for attention, 2 (d^2 + d O) per
+    token for the projector.  Returns (total, tcgen05-GEMM part)."""
+    C, d, F, O, L = (cfg.downsample_hidden_size, cfg.d_model, cfg.encoder_ffn_dim,
+                     cfg.output_dim, cfg.encoder_layers)
+    conv1 = conv23 = conv_out = 0
+    for n in lens:
+        for s in range(0, n, 100):
+            v = min(100, n - s)
+            f1 = _half(v)
+            f2 = _half(f1)
+            f3 = _half(f2)
+            conv1 += 2 * C * 9 * 64 * f1
+            conv23 += 2 * C * 9 * C * (32 * f2 + 16 * f3)
+            conv_out += 2 * f3 * 16 * C * d
+    T = cu[-1]
+    layers = L * 2 * (4 * d * d + 2 * d * F) * T
+    attn = L * 4 * d * sum((b - a) ** 2 for a, b in zip(cu[:-1], cu[1:]))
+    proj = 2 * (d * d + d * O) * T
+    gemm = conv23 + conv_out + layers + proj
+    return gemm + conv1 + attn, gemm
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons sampled through NVML every 5 ms
+    in a background thread while the timed region runs."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device):
+        import threading
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            h = None
+            try:
+                p = __import__("torch").cuda.get_device_properties(torch_device)
+                h = N.nvmlDeviceGetHandleByPciBusId(
+                    f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0")
+            except Exception:
+                h = N.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.N, self.h = N, h
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+            get_r = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                N.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self._stop.is_set():
+                    self.samples.append(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+                    r = get_r(h)
+                    for bit, name in self.REASONS.items():
+                        if r & bit:
+                            self.reasons.add(name)
+                    self._stop.wait(0.005)
+            self.t = threading.Thread(target=loop, daemon=True)
+            self.t.start()
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.t = None
+            self.error = str(e)
+
+    def stop(self):
+        if self.t is None:
+            return {"error": getattr(self, "error", "nvml unavailable")}
+        self._stop.set()
+        self.t.join()
+        sm = self.samples
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(sm) if sm else None, "reasons": sorted(self.reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU oracle ----
+def cpu_oracle_run(cfg, w, feats, lens):
+    import oracle as O
+    t0 = time.perf_counter()
+    O.forward(cfg, w, feats, lens, dtype=np.float32)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(workload, lens, seconds_wanted=30.0):
+    """A bounded sample of the workload for the CPU oracle: its first requests
+    until about `seconds_wanted` of audio (clipped to a whole number of windows)."""
+    out, tot = [], 0
+    for n in lens:
+        take = min(n, int(seconds_wanted * 100) - tot)
+        if take <= 0:
+            break
+        out.append(take)
+        tot += take
+    return out
+
+
+def reference_arm(args, rank, world):
+    """The oracle as it stands, timed on the host cores; each step encodes one
+    8 s window of the workload's first request."""
+    if rank != 0:
+        return
+    cfg = S.WORKLOADS[args.workload]
+    lens_all = S.request_lengths(args.workload)
+    w = S.weights(cfg)
+    lens = [min(lens_all[0], cfg.n_window_infer)]
+    feats = S.features(lens)
+    for _ in range(args.warmup):
+        cpu_oracle_run(cfg, w, feats, lens)
+    ts = [cpu_oracle_run(cfg, w, feats, lens) for _ in range(args.steps)]
+    audio = sum(lens) / 100.0
+    value = audio * len(ts) / sum(ts)
+    cores = len(os.sched_getaffinity(0))
+    sample = f"{lens[0]} frames (one attention window) of request 0 per step, numpy fp32"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(ts) / len(ts),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": args.workload},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm ----
+def our_arm(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from audio_encoder_aut_b200 import _lib as A
+    from audio_encoder_aut_b200.encoder import Encoder
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = S.WORKLOADS[args.workload]
+    lens = S.request_lengths(args.workload)
+    w = S.weights(cfg)
+    feats = S.features(lens, seed=S.SEED_FEATURES + rank)
+    enc = Encoder(cfg, w, local_rank)
+    tpr, cu, T, nW, nch = enc.plan(lens)
+    audio_s = sum(lens) / 100.0
+    fd = enc.features_to_device(feats)
+    out = torch.empty((T, cfg.output_dim), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, k):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(k)]
+        barrier()
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    for _ in range(args.warmup):
+        enc.encode(fd, lens, out=out)
+    torch.cuda.synchronize()
+    assert enc.check() == A.AUT_OK
+
+    sampler = ClockSampler(dev)
+    step_ms = timed(lambda: enc.encode(fd, lens, out=out), args.steps)
+    clocks = sampler.stop()
+    status = enc.check()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / args.steps
+    value = world * audio_s * args.steps / (total_ms / 1e3)
+    tokens_s = world * T * args.steps / (total_ms / 1e3)
+    flops, gemm_flops = credited_flops(cfg, lens, cu)
+    pk, pk_sus, hbm, pk_src = peaks()
+
+    # Per-kernel breakdown from traced steps (events recorded between launches).
+    cap = 4096
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    for e in events:  # torch creates the CUDA event on first record
+        e.record(stream)
+    torch.cuda.synchronize()
+    ev_ptrs = (A.c_void_p * cap)(*[e.cuda_event for e in events])
+    kinds = (A.c_int32 * cap)()
+    trace = A.aut_trace(ev_ptrs, cap, 0, kinds)
+    per_kind = {}
+    launches = 0
+    n_trace = max(1, min(3, args.steps))
+    for _ in range(n_trace):
+        flush.zero_()
+        start = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        enc.encode(fd, lens, out=out, trace=trace)
+        torch.cuda.synchronize()
+        launches = trace.count
+        prev = start
+        for i in range(min(trace.count, cap)):
+            k = A.KERNEL_KINDS[kinds[i]]
+            per_kind.setdefault(k, []).append(prev.elapsed_time(events[i]))
+            prev = events[i]
+    kind_ms = {k: sum(v) / n_trace for k, v in per_kind.items()}
+    gemm_launches = sum(len(v) for k, v in per_kind.items() if k in A.GEMM_KINDS) / n_trace
+    gemm_ms = sum(kind_ms[k] for k in kind_ms if k in A.GEMM_KINDS)
+    gemm_avg_ms = gemm_ms / gemm_launches
+    achieved = gemm_flops / gemm_launches / (gemm_avg_ms / 1e3) / 1e12
+
+    # End to end through the public API: pinned host features in, result back out.
+    h_feats = fd.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        fd.copy_(h_feats, non_blocking=True)
+        enc.encode(fd, lens, out=out)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms = timed(e2e_step, args.steps)
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = world * audio_s * args.steps / (e2e_total / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = oracle_sample(args.workload, lens, args.cpu_sample_seconds)
+        sfeats = S.features(sample, seed=S.SEED_FEATURES)
+        dt = cpu_oracle_run(cfg, w, sfeats, sample)
+        cpu = {"value": (sum(sample) / 100.0) / dt, "unit": UNIT,
+               "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"first {len(sample)} request(s) of the workload cut to "
+                         f"{sum(sample)} frames ({sum(sample) / 100:.0f} s audio), numpy fp32, "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        q = sorted(step_ms)
+        pct = lambda p: q[min(len(q) - 1, int(math.ceil(p / 100 * len(q))) - 1)]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "requests": len(lens), "frames": sum(lens),
+                       "audio_seconds": audio_s, "total_tokens": T, "windows": nW,
+                       "chunks": nch, "d_model": cfg.d_model, "layers": cfg.encoder_layers,
+                       "l2": "256 MiB buffer written between timed steps (outside the events)",
+                       "parallelism": f"dp{world} (weak: one batch per GPU)"},
+            "tokens_per_s": tokens_s,
+            "tflops": flops / (ms / 1e3) / 1e12,
+            "pct_bf16_peak": 100 * flops / (ms / 1e3) / 1e12 / pk,
+            "pct_bf16_peak_sustained": 100 * flops / (ms / 1e3) / 1e12 / pk_sus,
+            "step_ms_p50_p95_p99": [pct(50), pct(95), pct(99)],
+            "credited_gflop_per_step": flops / 1e9,
+            "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (all tcgen05 GEMM launches)",
+                         "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                         "frac": achieved / pk, "peak_source": f"{pk_src} bf16 burst",
+                         "peak_sustained": pk_sus, "launches_per_step": gemm_launches,
+                         "avg_launch_ms": gemm_avg_ms, "traffic": None},
+            "kernel_ms_per_step": {k: round(v, 4) for k, v in sorted(kind_ms.items(), key=lambda x: -x[1])},
+            "e2e": {"value": e2e_value, "unit": UNIT,
+                    "h2d_bytes_per_step": h_feats.numel() * h_feats.element_size(),
+                    "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
+                    "ms_per_step": e2e_total / args.steps},
+            "gpu_launches": launches * args.steps,
+            "device_status": A.status_string(status),
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="omni_16req", choices=sorted(S.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=60.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        our_arm(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

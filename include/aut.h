@@ -15,8 +15,8 @@
  *     addresses on the current CUDA device.
  *   - Streams: device work is enqueued on `stream` and returns before it ends
  *     (asynchronous); host buffers passed in are read before the call returns.
- *   - Types: every parameter, the features and the encoder output are bf16
- *     (stored as 16-bit words); the residual stream ("hidden") is fp32.
+ *   - Types: every parameter and the features are bf16 (stored as 16-bit
+ *     words); the residual stream ("hidden") and the encoder output are fp32.
  *   - Layouts are row-major.  Linear weights follow PyTorch: [out, in].  Conv
  *     weights are [C_out, C_in, 3, 3].  The fused qkv weight stacks q, k, v on
  *     dim 0 ([3 d, d]) and head h uses columns [h*hd, (h+1)*hd) of each.
@@ -87,8 +87,12 @@ typedef struct {
     const void *ln_post_w, *ln_post_b, *proj1_w, *proj1_b, *proj2_w, *proj2_b;
     /* Filled by aut_prepare_weights, NULL in caller-built structs: kernel-layout
      * copies of conv2_w/conv3_w ([C][9][C]: out, tap, in), conv_out_w
-     * ([d][16*C]: index f*C + c) and the fp32 sinusoid table [13][d]. */
+     * ([d][16*C]: index f*C + c), the fp32 sinusoid table [13][d], and the
+     * projector weights repeated along K ([d][2d], [output_dim][2d]) for the
+     * two-term (hi + lo bf16) projector operands. */
     const void *conv2_w_tap, *conv3_w_tap, *conv_out_w_fc, *pos_table;
+    const void *proj1_w_dup, *proj2_w_dup;
+    const void *o_w_dup; /* [layers][d][2d]: every layer's o_proj weight repeated along K */
 } aut_weights;
 
 /* aut_encoder page, AuTEncoder.layout / AuTEncoderConfig.tokens_for_frames /
@@ -115,10 +119,10 @@ size_t aut_prepared_bytes(const aut_config *cfg);
 /* One-time weight preparation (cubic.dev "Audio Encoder Component", Weight
  * Transposition: conv weights are re-laid-out channel-last for the kernels).
  * Writes into `dst` (device, dst_bytes >= aut_prepared_bytes) the tap-major conv2
- * and conv3 weights, conv_out's columns reordered to the stem's output order and
+ * and conv3 weights, conv_out's columns reordered to the stem's output order,
  * the sinusoid table (aut_encoder page, module docstring: the same 13 positions
- * for every chunk).  Copies `src` into `*prepared` and points the four prepared
- * fields into `dst`.  Asynchronous on `stream`; src stays owned by the caller and
+ * for every chunk) and the K-repeated o_proj and projector weights.  Copies
+ * `src` into `*prepared` and points the seven prepared fields into `dst`.  Asynchronous on `stream`; src stays owned by the caller and
  * must stay alive while `prepared` is used. */
 aut_status aut_prepare_weights(const aut_config *cfg, const aut_weights *src, void *dst,
                                size_t dst_bytes, aut_weights *prepared, aut_stream_t stream);
@@ -126,13 +130,49 @@ aut_status aut_prepare_weights(const aut_config *cfg, const aut_weights *src, vo
 /* aut_encoder page, AuTEncoder.forward: features -> [total_tokens, output_dim].
  * features: device bf16 [n_req, mel_bins, T_max], time fastest; frames at or
  * after feature_lens[r] are treated as zero whatever the buffer holds.
- * feature_lens: HOST int32 [n_req], each in [0, T_max].  out: device bf16
+ * feature_lens: HOST int32 [n_req], each in [0, T_max].  out: device fp32
  * [total_tokens, output_dim], rows in packed order (requests in input order,
  * tokens in time order).  workspace: device, ws_bytes >= aut_workspace_bytes.
  * `prepared` comes from aut_prepare_weights. */
 aut_status aut_encode(const aut_config *cfg, const aut_weights *prepared, const void *features,
                       int32_t T_max, const int32_t *feature_lens, int32_t n_req, void *out,
                       void *workspace, size_t ws_bytes, aut_stream_t stream);
+
+/* Kernel kinds reported by aut_encode_traced. */
+typedef enum {
+    AUT_K_UPLOAD = 0,    /* plan tables to the device */
+    AUT_K_ZERO_PADS = 1, /* zero borders of conv3's input planes */
+    AUT_K_CONV1 = 2,
+    AUT_K_CONV2 = 3,
+    AUT_K_CONV3 = 4,
+    AUT_K_CONV_OUT = 5,  /* conv_out + positions + packing */
+    AUT_K_LAYERNORM = 6,
+    AUT_K_QKV = 7,
+    AUT_K_ATTENTION = 8,
+    AUT_K_O_PROJ = 9,
+    AUT_K_FC1 = 10,
+    AUT_K_FC2 = 11,
+    AUT_K_PROJ1 = 12,
+    AUT_K_PROJ2 = 13
+} aut_kernel_kind;
+
+/* Per-kernel trace, the CUDA-event timing of each stage.  events: caller-created
+ * cudaEvent_t handles (NULL with capacity 0 to only count); kinds: int32
+ * [capacity] or NULL.  The library records events[i] on the stream right after
+ * its i-th kernel launch and stores the kernel's aut_kernel_kind in kinds[i];
+ * count receives the number of kernels launched (even beyond capacity). */
+typedef struct {
+    void **events;
+    int32_t capacity;
+    int32_t count;
+    int32_t *kinds;
+} aut_trace;
+
+/* aut_encode with a per-kernel trace (trace may be NULL). */
+aut_status aut_encode_traced(const aut_config *cfg, const aut_weights *prepared,
+                             const void *features, int32_t T_max, const int32_t *feature_lens,
+                             int32_t n_req, void *out, void *workspace, size_t ws_bytes,
+                             aut_stream_t stream, aut_trace *trace);
 
 /* aut_encoder page, AuTEncoder.frontend: features -> packed chunk embeddings
  * x0, device fp32 [total_tokens, d_model].  with_positions = 0 leaves out the
@@ -147,7 +187,7 @@ aut_status aut_frontend(const aut_config *cfg, const aut_weights *prepared, cons
  * over a packed sequence.  hidden: device fp32 [total_tokens, d_model], the
  * residual stream, updated in place by layers [0, n_layers).  cu_seqlens: HOST
  * int32 [num_windows + 1], non-decreasing from 0 to total_tokens, every window at
- * most 128 tokens.  If out (device bf16 [total_tokens, output_dim]) is not NULL,
+ * most 128 tokens.  If out (device fp32 [total_tokens, output_dim]) is not NULL,
  * the final LayerNorm and projector run after the layers and write it. */
 aut_status aut_encode_packed(const aut_config *cfg, const aut_weights *prepared, void *hidden,
                              int32_t total_tokens, const int32_t *cu_seqlens,
@@ -158,7 +198,8 @@ aut_status aut_encode_packed(const aut_config *cfg, const aut_weights *prepared,
  * fused qkv_proj of the aut_encoder page, o_proj, fc1/fc2 of the FFN, the
  * projector), exposed for kernel-level checks.  x: device bf16 [M, K]; w: device
  * bf16 [N, K]; bias: device bf16 [N] or NULL.  epilogue 0: y bf16 [M, N] =
- * acc + b; 1: y bf16 = GELU(acc + b); 2: y fp32 [M, N] += acc + b (residual add).
+ * acc + b; 1: y bf16 = GELU(acc + b); 2: y fp32 [M, N] += acc + b (residual add);
+ * 3: y fp32 [M, N] = acc + b.
  * K must be a multiple of 64 and N a multiple of 16.  status: device int32 word
  * for device-side faults (may be NULL).  timeout_ms bounds every pipeline wait
  * (0 = default of 4000 ms).  fault_inject = 1 makes the first block skip its first
@@ -178,7 +219,9 @@ aut_status aut_layernorm(const void *x, const void *gamma, const void *beta, voi
 /* Window attention (aut_encoder page, AuTAttention; openarchlab "1A . AuT Audio
  * Encoder", section 3: non-causal attention limited to each cu_seqlens segment):
  * for every segment and head, softmax(Q K^T / sqrt(hd)) V.  qkv: device bf16
- * [T, 3 d] (q | k | v); out: device bf16 [T, d].  cu_seqlens: HOST int32
+ * [T, 3 d] (q | k | v); out: device bf16 [T, 2 d], each row [hi | lo] with
+ * hi = bf16(o) and lo = bf16(o - hi), so hi + lo carries o to about 16
+ * significant bits (P is likewise applied as two bf16 terms).  cu_seqlens: HOST int32
  * [num_windows + 1], every window at most 128 tokens.  workspace: device, at
  * least 4 * (num_windows + 1) bytes (the uploaded cu_seqlens). */
 aut_status aut_window_attention(const void *qkv, void *out, int32_t T, int32_t d, int32_t heads,

@@ -6,7 +6,7 @@ import pytest
 
 import aut_synth as S
 import oracle as O
-from gpu_util import assert_rows_close
+from gpu_util import assert_bf16_output_close, assert_rows_close
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -59,7 +59,23 @@ def test_linear_matches_definition(M, N, K, epi):
         # fp32 output: only accumulation-order error
         np.testing.assert_allclose(got, ref, rtol=0, atol=2e-3 * np.sqrt(K / 64))
     else:
-        assert_rows_close(got, ref, f"linear {M}x{N}x{K} epi {epi}")
+        assert_bf16_output_close(got, ref, f"linear {M}x{N}x{K} epi {epi}")
+        assert_rows_close(got, ref, f"linear {M}x{N}x{K} epi {epi}", rel_max=3e-2)
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 1280, 1280), (31, 2048, 1280), (4000, 1024, 896)])
+def test_linear_fp32_output(M, N, K):
+    x = _rand((M, K), 1)
+    w = _rand((N, K), 2, 0.05)
+    b = _rand((N,), 3, 0.1)
+    ref = x.astype(np.float64) @ w.astype(np.float64).T + b
+    xd, wd, bd = _dev(x, torch.bfloat16), _dev(w, torch.bfloat16), _dev(b, torch.bfloat16)
+    yd = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    st = A.aut_linear(xd.data_ptr(), wd.data_ptr(), bd.data_ptr(), yd.data_ptr(), M, N, K,
+                      A.EPI_F32, None, 0, 0, _stream())
+    assert st == A.AUT_OK
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(yd.cpu().numpy(), ref, rtol=0, atol=2e-3 * np.sqrt(K / 64))
 
 
 def test_linear_no_bias_and_structured_inputs():
@@ -85,13 +101,13 @@ def test_layernorm_matches_oracle(T, d):
     g = S.round_bf16(1 + 0.1 * rng.standard_normal(d).astype(np.float32))
     b = S.round_bf16(0.1 * rng.standard_normal(d).astype(np.float32))
     y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
-    st = A.aut_layernorm(_dev(x, torch.float32).data_ptr(), _dev(g, torch.bfloat16).data_ptr(),
-                         _dev(b, torch.bfloat16).data_ptr(), y.data_ptr(), T, d, 1e-5, _stream())
+    xd, gd, bd = _dev(x, torch.float32), _dev(g, torch.bfloat16), _dev(b, torch.bfloat16)
+    st = A.aut_layernorm(xd.data_ptr(), gd.data_ptr(), bd.data_ptr(), y.data_ptr(), T, d, 1e-5,
+                         _stream())
     assert st == A.AUT_OK
     torch.cuda.synchronize()
     ref = O.layer_norm(x.astype(np.float64), g, b, 1e-5)
-    assert_rows_close(y.float().cpu().numpy(), ref, "layernorm")
-    np.testing.assert_allclose(y.float().cpu().numpy(), ref, rtol=1e-2, atol=1e-2)
+    assert_bf16_output_close(y.float().cpu().numpy(), ref, "layernorm")
 
 
 ATTN_CASES = [
@@ -111,14 +127,22 @@ def test_window_attention_matches_oracle(heads, hd, lens):
         cu.append(cu[-1] + n)
     T = cu[-1]
     qkv = _rand((T, 3 * d), 11, 1.0)
-    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((T, 2 * d), dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
-    st = A.aut_window_attention(_dev(qkv, torch.bfloat16).data_ptr(), out.data_ptr(), T, d, heads,
-                                cu, ws.data_ptr(), ws.numel(), _stream())
+    qd = _dev(qkv, torch.bfloat16)
+    st = A.aut_window_attention(qd.data_ptr(), out.data_ptr(), T, d, heads, cu, ws.data_ptr(),
+                                ws.numel(), _stream())
     assert st == A.AUT_OK
     torch.cuda.synchronize()
     ref = O.window_attention(qkv.astype(np.float64), cu, heads)
-    assert_rows_close(out.float().cpu().numpy(), ref, "window attention")
+    o = out.float().cpu().numpy().astype(np.float64)
+    hi, lo = o[:, :d], o[:, d:]
+    # hi alone: the bf16 rounding of O (2^-8 |o|) on top of a near-exact O
+    vmax = np.abs(qkv[:, 2 * d:]).max()
+    assert_bf16_output_close(hi, ref, "window attention (hi)", atol=1e-4 * vmax)
+    # hi + lo: P and O carried as two bf16 terms; what is left is fp32
+    # accumulation and the exp2 evaluation (relative ~1e-6), bounded here by 1e-4.
+    np.testing.assert_allclose(hi + lo, ref, rtol=1e-4, atol=1e-4 * vmax)
 
 
 def test_pipeline_wait_timeout_returns_status_and_gpu_stays_usable():
