@@ -16,6 +16,7 @@ AUT_OK, AUT_ERR_INVALID_ARG, AUT_ERR_UNSUPPORTED, AUT_ERR_WORKSPACE, AUT_ERR_CUD
     AUT_ERR_TIMEOUT = range(6)
 
 EPI_BF16, EPI_BF16_GELU, EPI_RESID_F32, EPI_F32 = 0, 1, 2, 3
+LINEAR_FAULT_INJECT, LINEAR_SINGLE_CTA = 1, 2
 
 KERNEL_KINDS = ["upload", "zero_pads", "conv1", "conv2", "conv3", "conv_out", "layernorm",
                 "qkv", "attention", "o_proj", "fc1", "fc2", "proj1", "proj2"]
@@ -207,9 +208,8 @@ def aut_encode_packed(cfg, prepared, hidden: int, total_tokens: int, cu_seqlens,
 
 
 def aut_linear(x: int, w: int, bias: int | None, y: int, M: int, N: int, K: int, epilogue: int,
-               status: int | None, timeout_ms: int, fault_inject: int, stream: int) -> int:
-    return lib().aut_linear(x, w, bias, y, M, N, K, epilogue, status, timeout_ms, fault_inject,
-                            stream)
+               status: int | None, timeout_ms: int, flags: int, stream: int) -> int:
+    return lib().aut_linear(x, w, bias, y, M, N, K, epilogue, status, timeout_ms, flags, stream)
 
 
 def aut_layernorm(x: int, gamma: int, beta: int, y: int, T: int, d: int, eps: float,

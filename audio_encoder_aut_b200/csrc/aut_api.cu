@@ -449,7 +449,7 @@ extern "C" aut_status aut_encode_packed(const aut_config *cfg, const aut_weights
 
 extern "C" aut_status aut_linear(const void *x, const void *w, const void *bias, void *y, int32_t M,
                                  int32_t N, int32_t K, int32_t epilogue, int32_t *status,
-                                 int32_t timeout_ms, int32_t fault_inject, aut_stream_t stream) {
+                                 int32_t timeout_ms, int32_t flags, aut_stream_t stream) {
     if (M < 0 || N <= 0 || K <= 0 || epilogue < 0 || epilogue > 3 || timeout_ms < 0)
         return AUT_ERR_INVALID_ARG;
     if (M > 0 && (!x || !w || !y)) return AUT_ERR_INVALID_ARG;
@@ -466,7 +466,8 @@ extern "C" aut_status aut_linear(const void *x, const void *w, const void *bias,
     L.epi = epilogue == 3 ? kEpiF32 : epilogue;
     L.status = reinterpret_cast<int *>(status);
     L.timeout_ns = timeout_ms ? (unsigned long long)timeout_ms * 1000000ull : kDefaultTimeoutNs;
-    L.fault_inject = fault_inject ? 1 : 0;
+    L.fault_inject = (flags & AUT_LINEAR_FAULT_INJECT) ? 1 : 0;
+    L.single_cta = (flags & AUT_LINEAR_SINGLE_CTA) != 0;
     return gemm_status(launch_linear(L, reinterpret_cast<cudaStream_t>(stream)));
 }
 

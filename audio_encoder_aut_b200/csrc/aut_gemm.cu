@@ -53,58 +53,90 @@ int sm_count() {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int BN>
+template <int BN, int CG>
 GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
                cudaStream_t st) {
-    using Cfg = GemmCfg<BN>;
+    using Cfg = GemmCfg<BN, CG>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return GemmStatus::kLaunch;
     if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_tc_kernel<BN, CG>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg::SMEM_BYTES) != cudaSuccess)
             return GemmStatus::kLaunch;
         attr_done[dev] = true;
     }
     const int tiles = args.num_m_tiles * args.num_n_tiles;
-    const int grid = std::min(tiles, sm_count());
-    gemm_tc_kernel<BN><<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta, tb, args);
-    return cudaGetLastError() == cudaSuccess ? GemmStatus::kOk : GemmStatus::kLaunch;
+    const int groups = std::min(tiles, sm_count() / CG);
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3(groups * CG);
+    lc.blockDim = dim3(kGemmThreads);
+    lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (CG == 2) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+    }
+    const cudaError_t e = cudaLaunchKernelEx(&lc, gemm_tc_kernel<BN, CG>, ta, tb, args);
+    return e == cudaSuccess ? GemmStatus::kOk : GemmStatus::kLaunch;
 }
 
-GemmStatus dispatch(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
-                    cudaStream_t st) {
+GemmStatus dispatch(int bn, int cg, const CUtensorMap &ta, const CUtensorMap &tb,
+                    const GemmArgs &args, cudaStream_t st) {
+    if (cg == 2) {
+        switch (bn) {
+            case 64: return run<64, 2>(ta, tb, args, st);
+            case 128: return run<128, 2>(ta, tb, args, st);
+            case 192: return run<192, 2>(ta, tb, args, st);
+            case 240: return run<240, 2>(ta, tb, args, st);
+            case 256: return run<256, 2>(ta, tb, args, st);
+            default: return GemmStatus::kBadShape;
+        }
+    }
     switch (bn) {
-        case 16: return run<16>(ta, tb, args, st);
-        case 32: return run<32>(ta, tb, args, st);
-        case 64: return run<64>(ta, tb, args, st);
-        case 128: return run<128>(ta, tb, args, st);
-        case 192: return run<192>(ta, tb, args, st);
-        case 240: return run<240>(ta, tb, args, st);
-        case 256: return run<256>(ta, tb, args, st);
+        case 16: return run<16, 1>(ta, tb, args, st);
+        case 32: return run<32, 1>(ta, tb, args, st);
+        case 64: return run<64, 1>(ta, tb, args, st);
+        case 128: return run<128, 1>(ta, tb, args, st);
+        case 192: return run<192, 1>(ta, tb, args, st);
+        case 240: return run<240, 1>(ta, tb, args, st);
+        case 256: return run<256, 1>(ta, tb, args, st);
         default: return GemmStatus::kBadShape;
     }
 }
 
-// Tile width for a plain GEMM: the candidate that divides N with the fewest
-// (waves x per-tile cost); wider tiles reuse each A tile over more columns.
-int choose_bn(int M, int N, int sms) {
+bool pair_ok(int bn) { return bn == 64 || bn == 128 || bn == 192 || bn == 240 || bn == 256; }
+
+// Tile shape for a plain GEMM: the (width, CTAs per MMA) with the fewest waves
+// x per-tile cost; a CTA pair streams a third less operand data per FLOP.
+void choose_tile(int M, int N, int sms, bool allow_pair, int *bn_out, int *cg_out) {
     static const int cand[] = {256, 128, 64, 32, 16};
-    const int mt = (M + 127) / 128;
-    int best = 0;
-    long best_cost = 0;
-    for (int bn : cand) {
-        if (N % bn) continue;
-        const long tiles = (long)mt * (N / bn);
-        const long waves = (tiles + sms - 1) / sms;
-        const long cost = waves * (bn + 32);
-        if (!best || cost < best_cost) {
-            best = bn;
-            best_cost = cost;
+    long best_cost = -1;
+    *bn_out = 0;
+    *cg_out = 1;
+    for (int cg = 1; cg <= 2; ++cg) {
+        if (cg == 2 && (!allow_pair || M <= 128)) continue;
+        for (int bn : cand) {
+            if (N % bn || (cg == 2 && !pair_ok(bn))) continue;
+            const long mt = (M + 128 * cg - 1) / (128 * cg);
+            const long tiles = mt * (N / bn);
+            const long slots = sms / cg;
+            const long waves = (tiles + slots - 1) / slots;
+            const long cost = waves * cg * 128 * (bn + 32) * (cg == 2 ? 5 : 6);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
+                *bn_out = bn;
+                *cg_out = cg;
+            }
         }
     }
-    return best;
 }
 
 }  // namespace
@@ -115,20 +147,21 @@ GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
         return GemmStatus::kBadShape;
     if (!aligned16(L.a) || !aligned16(L.w) || !aligned16(L.out) || (L.bias && !aligned16(L.bias)))
         return GemmStatus::kBadShape;
-    const int bn = choose_bn(L.M, L.N, sm_count());
+    int bn = 0, cg = 1;
+    choose_tile(L.M, L.N, sm_count(), L.fault_inject == 0 && !L.single_cta, &bn, &cg);
     if (!bn) return GemmStatus::kBadShape;
     CUtensorMap ta, tb;
     const cuuint64_t da[2] = {(cuuint64_t)L.K, (cuuint64_t)L.M};
     const cuuint64_t sa[1] = {(cuuint64_t)L.K * 2};
     const cuuint32_t ba[2] = {64, 128};
     const cuuint64_t db[2] = {(cuuint64_t)L.K, (cuuint64_t)L.N};
-    const cuuint32_t bb[2] = {64, (cuuint32_t)bn};
+    const cuuint32_t bb[2] = {64, (cuuint32_t)(bn / cg)};
     if (!make_map(&ta, 2, L.a, da, sa, ba) || !make_map(&tb, 2, L.w, db, sa, bb))
         return GemmStatus::kTensorMap;
     GemmArgs args{};
     args.M = L.M;
     args.N = L.N;
-    args.num_m_tiles = (L.M + 127) / 128;
+    args.num_m_tiles = (L.M + 128 * cg - 1) / (128 * cg);
     args.num_n_tiles = L.N / bn;
     args.num_k_blocks = L.K / 64;
     args.conv = 0;
@@ -142,7 +175,7 @@ GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
     args.status = L.status;
     args.timeout_ns = L.timeout_ns;
     args.fault_inject = L.fault_inject;
-    return dispatch(bn, ta, tb, args, st);
+    return dispatch(bn, cg, ta, tb, args, st);
 }
 
 GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
@@ -151,6 +184,7 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     if (!bn || L.rows_per_tile * L.out_cols > 128) return GemmStatus::kBadShape;
     if (!aligned16(L.planes) || !aligned16(L.w_tap) || !aligned16(L.out) || !aligned16(L.bias))
         return GemmStatus::kBadShape;
+    const int cg = (!L.single_cta && pair_ok(bn)) ? 2 : 1;
     const long rows_total = (long)L.chunks * L.chunk_rows;
     CUtensorMap ta, tb;
     const cuuint64_t da[4] = {(cuuint64_t)L.C, (cuuint64_t)L.cols_in, (cuuint64_t)rows_total, 4};
@@ -159,13 +193,14 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     const cuuint32_t ba[4] = {64, (cuuint32_t)L.out_cols, (cuuint32_t)L.rows_per_tile, 1};
     const cuuint64_t db[3] = {(cuuint64_t)L.C, 9, (cuuint64_t)L.C};
     const cuuint64_t sb[2] = {(cuuint64_t)L.C * 2, (cuuint64_t)9 * L.C * 2};
-    const cuuint32_t bb[3] = {64, 1, (cuuint32_t)bn};
+    const cuuint32_t bb[3] = {64, 1, (cuuint32_t)(bn / cg)};
     if (!make_map(&ta, 4, L.planes, da, sa, ba) || !make_map(&tb, 3, L.w_tap, db, sb, bb))
         return GemmStatus::kTensorMap;
     GemmArgs args{};
     args.M = (int)rows_total;
     args.N = L.C;
-    args.num_m_tiles = (int)((rows_total + L.rows_per_tile - 1) / L.rows_per_tile);
+    const long slot_rows = (long)L.rows_per_tile * cg;
+    args.num_m_tiles = (int)((rows_total + slot_rows - 1) / slot_rows);
     args.num_n_tiles = L.C / bn;
     args.conv = 1;
     args.conv_rows = L.rows_per_tile;
@@ -183,7 +218,7 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     args.dst_cols = L.dst_cols;
     args.status = L.status;
     args.timeout_ns = L.timeout_ns;
-    return dispatch(bn, ta, tb, args, st);
+    return dispatch(bn, cg, ta, tb, args, st);
 }
 
 }  // namespace aut

@@ -61,11 +61,14 @@ struct GemmArgs {
     int fault_inject;
 };
 
-template <int BN>
+// BN: tile width of one MMA (N).  CG: CTAs per MMA (1, or 2 for a CTA pair
+// whose MMA is M = 256: each CTA holds 128 rows of A and BN / 2 rows of B).
+template <int BN, int CG>
 struct GemmCfg {
     static constexpr int BM = 128, BK = 64;
     static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_ROWS = BN / CG;
+    static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES_FIT = 196608 / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
@@ -76,7 +79,8 @@ struct GemmCfg {
                                                        : 512;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + BAR_BYTES;
-    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M = 128");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
+    static_assert(B_ROWS % 8 == 0, "each CTA holds whole 8-row swizzle atoms of B");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay aligned");
 };
 
@@ -123,11 +127,11 @@ AUT_DEV void add_bias16(float (&v)[16], const __nv_bfloat16 *bias, int n0) {
     }
 }
 
-template <int BN>
+template <int BN, int CG>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs args) {
-    using Cfg = GemmCfg<BN>;
+    using Cfg = GemmCfg<BN, CG>;
     constexpr int STAGES = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -143,6 +147,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;  // 0 issues the MMAs
+    const int group = blockIdx.x / CG, n_groups = gridDim.x / CG;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full + s, 1);
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull + a, 1);
-            mbar_init(tempty + a, kEpilogueWarps);
+            mbar_init(tempty + a, kEpilogueWarps * CG);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -161,11 +167,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (CG == 2) {
+            tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    if constexpr (CG == 2)
+        cluster_sync();  // barriers of both CTAs initialised before any remote use
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     volatile int *abort_v = abort_flag;
@@ -175,11 +190,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer --
+            // Both CTAs of a pair load their own A rows and B half; the loads of
+            // both complete on the even CTA's `full` barrier, which the even CTA
+            // arms with the pair's byte count.
             int stage = 0;
             uint32_t phase = 0, issued = 0, parity = 0;
             bool ok = true, skip = args.fault_inject != 0 && blockIdx.x == 0;
-            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+            for (int tile = group; ok && tile < total_tiles; tile += n_groups) {
                 const int n_blk = tile % args.num_n_tiles, m_blk = tile / args.num_n_tiles;
+                const int m_slot = m_blk * CG + (int)rank;  // this CTA's 128-row slot
+                const int b_row = n_blk * BN + (int)rank * Cfg::B_ROWS;
                 for (int kb = 0; kb < args.num_k_blocks; ++kb) {
                     if (!mbar_wait(empty + stage, phase ^ 1u, abort_v, lim)) {
                         ok = false;
@@ -190,10 +210,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     } else {
                         uint8_t *a_dst = sA + stage * Cfg::A_BYTES;
                         uint8_t *b_dst = sB + stage * Cfg::B_BYTES;
+                        const uint32_t a_bytes =
+                            args.conv ? 128u * args.conv_rows * args.conv_cols : (uint32_t)Cfg::A_BYTES;
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(full + stage, CG * (a_bytes + Cfg::B_BYTES));
                         if (!args.conv) {
-                            mbar_arrive_expect_tx(full + stage, Cfg::A_BYTES + Cfg::B_BYTES);
-                            tma_load_2d(a_dst, &tmA, full + stage, kb * 64, m_blk * 128);
-                            tma_load_2d(b_dst, &tmB, full + stage, kb * 64, n_blk * BN);
+                            if constexpr (CG == 2) {
+                                const uint32_t bar = map_to_rank(full + stage, 0);
+                                tma_load_2d_pair(a_dst, &tmA, bar, kb * 64, m_slot * 128);
+                                tma_load_2d_pair(b_dst, &tmB, bar, kb * 64, b_row);
+                            } else {
+                                tma_load_2d(a_dst, &tmA, full + stage, kb * 64, m_slot * 128);
+                                tma_load_2d(b_dst, &tmB, full + stage, kb * 64, b_row);
+                            }
                         } else {
                             const int tap = kb / args.conv_cblocks;
                             const int cb = kb - tap * args.conv_cblocks;
@@ -203,11 +232,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             // counting the leading zero row.  Same for kw along columns.
                             const int plane = (kh == 1 ? 0 : 2) + (kw == 1 ? 0 : 1);
                             const int dh = kh == 0 ? 0 : 1, dw = kw == 0 ? 0 : 1;
-                            const uint32_t a_bytes = 128u * args.conv_rows * args.conv_cols;
-                            mbar_arrive_expect_tx(full + stage, a_bytes + Cfg::B_BYTES);
-                            tma_load_4d(a_dst, &tmA, full + stage, cb * 64, dw,
-                                        m_blk * args.conv_rows + dh, plane);
-                            tma_load_3d(b_dst, &tmB, full + stage, cb * 64, tap, n_blk * BN);
+                            const int vrow = m_slot * args.conv_rows + dh;
+                            if constexpr (CG == 2) {
+                                const uint32_t bar = map_to_rank(full + stage, 0);
+                                tma_load_4d_pair(a_dst, &tmA, bar, cb * 64, dw, vrow, plane);
+                                tma_load_3d_pair(b_dst, &tmB, bar, cb * 64, tap, b_row);
+                            } else {
+                                tma_load_4d(a_dst, &tmA, full + stage, cb * 64, dw, vrow, plane);
+                                tma_load_3d(b_dst, &tmB, full + stage, cb * 64, tap, b_row);
+                            }
                         }
                         issued |= 1u << stage;
                         parity = (parity & ~(1u << stage)) | (phase << stage);
@@ -219,18 +252,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
             if (!ok) gemm_signal_abort(args, abort_v);
-            // The last load issued on every stage has landed before the block may exit.
-            for (int s = 0; s < STAGES; ++s)
-                if (issued >> s & 1u) mbar_wait(full + s, parity >> s & 1u, nullptr, lim);
+            if (rank == 0) {
+                // The last load issued on every stage has landed before the block may exit.
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued >> s & 1u) mbar_wait(full + s, parity >> s & 1u, nullptr, lim);
+            } else if (!ok) {
+                // The odd CTA's loads complete on the even CTA's barriers; after a
+                // failure give its copies in flight time to land before exiting.
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 200000ull) {
+                }
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             // -------------------------------------------------- MMA issuer --
-            constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+            constexpr uint32_t idesc = idesc_bf16_f32(128 * CG, BN);
+            constexpr uint16_t kPair = 0x3;
             int stage = 0, it = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
+            for (int tile = group; ok && tile < total_tiles; tile += n_groups, ++it) {
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!mbar_wait(tempty + acc, acc_phase ^ 1u, abort_v, lim)) {
@@ -248,21 +290,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint64_t a_desc = smem_desc_sw128(sA + stage * Cfg::A_BYTES);
                     const uint64_t b_desc = smem_desc_sw128(sB + stage * Cfg::B_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // K = 16 per MMA: +32 bytes in the row
-                        tc_mma_bf16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
-                                    (kb | kk) != 0);
-                    tc_commit(empty + stage);
+                    for (int kk = 0; kk < 4; ++kk) {  // K = 16 per MMA: +32 bytes in the row
+                        if constexpr (CG == 2)
+                            tc_mma_bf16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
+                                             (kb | kk) != 0);
+                        else
+                            tc_mma_bf16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
+                                        (kb | kk) != 0);
+                    }
+                    if constexpr (CG == 2)
+                        tc_commit_pair(empty + stage, kPair);
+                    else
+                        tc_commit(empty + stage);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit(tfull + acc);
+                if constexpr (CG == 2)
+                    tc_commit_pair(tfull + acc, kPair);
+                else
+                    tc_commit(tfull + acc);
             }
             if (!ok) gemm_signal_abort(args, abort_v);
             // Every MMA this thread issued has completed before TMEM is released.
-            tc_commit(mma_done);
+            if constexpr (CG == 2)
+                tc_commit_pair(mma_done, 0x1);
+            else
+                tc_commit(mma_done);
             mbar_wait(mma_done, 0, nullptr, lim);
         }
     } else {
@@ -276,7 +332,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         constexpr int NC = BN / 16;
         int it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+        const uint32_t tempty_even = CG == 2 ? map_to_rank(tempty, 0) : 0;
+        for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             if (!mbar_wait(tfull + acc, acc_phase, abort_v, lim)) {
@@ -284,7 +341,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int n_blk = tile % args.num_n_tiles, m_blk = tile / args.num_n_tiles;
+            const int n_blk = tile % args.num_n_tiles;
+            const int m_blk = (tile / args.num_n_tiles) * CG + (int)rank;  // 128-row slot
 
             // Where this thread's accumulator row goes.
             bool valid = true;
@@ -412,15 +470,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty + acc);
+            if (lane == 0) {
+                if constexpr (CG == 2)
+                    mbar_arrive_cluster(tempty_even + acc * 8);
+                else
+                    mbar_arrive(tempty + acc);
+            }
         }
         if (!ok && lane == 0) gemm_signal_abort(args, abort_v);
     }
 
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    __syncwarp();
+    if constexpr (CG == 2) {
+        cluster_sync();  // both CTAs done with TMEM and with each other's barriers
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+        }
+    } else {
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+        }
     }
 }
 

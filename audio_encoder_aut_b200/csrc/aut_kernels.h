@@ -58,6 +58,7 @@ struct LinearLaunch {
     int *status;
     unsigned long long timeout_ns;
     int fault_inject;
+    bool single_cta = false;  // force one CTA per MMA (no CTA pairs)
 };
 GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st);
 
@@ -77,6 +78,7 @@ struct ConvLaunch {
     int dst_plane_rows, dst_chunk_rows, dst_cols;  // kEpiConvPlanes destination geometry
     int *status;
     unsigned long long timeout_ns;
+    bool single_cta = false;
 };
 GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st);
 

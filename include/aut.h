@@ -202,12 +202,15 @@ aut_status aut_encode_packed(const aut_config *cfg, const aut_weights *prepared,
  * 3: y fp32 [M, N] = acc + b.
  * K must be a multiple of 64 and N a multiple of 16.  status: device int32 word
  * for device-side faults (may be NULL).  timeout_ms bounds every pipeline wait
- * (0 = default of 4000 ms).  fault_inject = 1 makes the first block skip its first
- * operand load so that its consumer's wait runs out (tests of the timeout path
- * only); 0 otherwise. */
+ * (0 = default of 4000 ms).  flags: AUT_LINEAR_FAULT_INJECT makes the first block
+ * skip its first operand load so that its consumer's wait runs out (tests of the
+ * timeout path only); AUT_LINEAR_SINGLE_CTA keeps every MMA on one SM (no CTA
+ * pairs); 0 for normal use. */
+#define AUT_LINEAR_FAULT_INJECT 1
+#define AUT_LINEAR_SINGLE_CTA 2
 aut_status aut_linear(const void *x, const void *w, const void *bias, void *y, int32_t M,
                       int32_t N, int32_t K, int32_t epilogue, int32_t *status,
-                      int32_t timeout_ms, int32_t fault_inject, aut_stream_t stream);
+                      int32_t timeout_ms, int32_t flags, aut_stream_t stream);
 
 /* LayerNorm with bias over the last dim (cubic.dev "Audio Encoder Component",
  * Transformer Encoder Layers): y = (x - mean) / sqrt(var + eps) * gamma + beta,

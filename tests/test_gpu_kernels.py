@@ -32,9 +32,10 @@ SHAPES = [(1, 64, 64), (31, 192, 64), (128, 256, 256), (300, 1280, 1280), (1000,
           (3000, 1280, 5120), (513, 2048, 1280), (45, 1024, 896)]
 
 
+@pytest.mark.parametrize("flags", [0, A.LINEAR_SINGLE_CTA], ids=["auto", "single_cta"])
 @pytest.mark.parametrize("M,N,K", SHAPES)
 @pytest.mark.parametrize("epi", [A.EPI_BF16, A.EPI_BF16_GELU, A.EPI_RESID_F32])
-def test_linear_matches_definition(M, N, K, epi):
+def test_linear_matches_definition(M, N, K, epi, flags):
     x = _rand((M, K), 1)
     w = _rand((N, K), 2, 0.05)
     b = _rand((N,), 3, 0.1)
@@ -50,7 +51,7 @@ def test_linear_matches_definition(M, N, K, epi):
         if epi == A.EPI_BF16_GELU:
             ref = O.gelu(ref)
     st = A.aut_linear(xd.data_ptr(), wd.data_ptr(), bd.data_ptr(), yd.data_ptr(), M, N, K, epi,
-                      status.data_ptr(), 0, 0, _stream())
+                      status.data_ptr(), 0, flags, _stream())
     assert st == A.AUT_OK
     torch.cuda.synchronize()
     assert int(status.item()) == 0
@@ -78,16 +79,18 @@ def test_linear_fp32_output(M, N, K):
     np.testing.assert_allclose(yd.cpu().numpy(), ref, rtol=0, atol=2e-3 * np.sqrt(K / 64))
 
 
-def test_linear_no_bias_and_structured_inputs():
+@pytest.mark.parametrize("M,N,K,flags", [(128, 256, 256, 0), (512, 256, 256, 0),
+                                         (512, 256, 256, A.LINEAR_SINGLE_CTA), (300, 240, 128, 0)])
+def test_linear_no_bias_and_structured_inputs(M, N, K, flags):
     """Identity-like A picks out rows of W: checks operand layout and K order exactly."""
-    M, N, K = 128, 256, 256
     x = np.zeros((M, K), np.float32)
     for i in range(M):
         x[i, (3 * i) % K] = 1.0
     w = _rand((N, K), 5)
+    xd, wd = _dev(x, torch.bfloat16), _dev(w, torch.bfloat16)
     yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    st = A.aut_linear(_dev(x, torch.bfloat16).data_ptr(), _dev(w, torch.bfloat16).data_ptr(),
-                      None, yd.data_ptr(), M, N, K, A.EPI_BF16, None, 0, 0, _stream())
+    st = A.aut_linear(xd.data_ptr(), wd.data_ptr(), None, yd.data_ptr(), M, N, K, A.EPI_BF16,
+                      None, 0, flags, _stream())
     assert st == A.AUT_OK
     torch.cuda.synchronize()
     ref = np.stack([w[:, (3 * i) % K] for i in range(M)])
@@ -155,7 +158,7 @@ def test_pipeline_wait_timeout_returns_status_and_gpu_stays_usable():
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     st = A.aut_linear(x.data_ptr(), w.data_ptr(), None, y.data_ptr(), M, N, K, A.EPI_BF16,
-                      status.data_ptr(), 200, 1, _stream())
+                      status.data_ptr(), 200, A.LINEAR_FAULT_INJECT, _stream())
     assert st == A.AUT_OK
     torch.cuda.synchronize()
     assert A.aut_check_status_word(status.data_ptr()) == A.AUT_ERR_TIMEOUT
