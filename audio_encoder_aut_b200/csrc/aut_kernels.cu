@@ -123,14 +123,16 @@ __global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int 
 // two passes (mean, then centred variance).  With `split`, the output row is
 // [hi | lo] (2 d wide): hi = bf16(y), lo = bf16(y - hi), so that a GEMM over
 // the doubled K against [W | W] sees y to about 16 significant bits.
+constexpr int kLnRowsPerBlock = 4;  // one warp per row
+
 template <int VPL>  // float4 per lane
-__global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict__ x,
+__global__ void __launch_bounds__(32 * kLnRowsPerBlock) layernorm_kernel(const float *__restrict__ x,
                                                         const bf16 *__restrict__ g,
                                                         const bf16 *__restrict__ bt,
                                                         bf16 *__restrict__ y, int T, int d,
                                                         float eps, int split) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.x * 8 + warp;
+    const int row = blockIdx.x * kLnRowsPerBlock + warp;
     if (row >= T) return;
     const int n4 = d >> 2;
     const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)row * d);
@@ -235,8 +237,7 @@ __global__ void __launch_bounds__(32 * kAttnWarps) window_attn_kernel(const bf16
                                                           float scale_log2e) {
     constexpr int LD = HD + 8;  // padded row: conflict-free ldmatrix
     extern __shared__ __align__(16) uint8_t attn_smem[];
-    bf16 *sQ = reinterpret_cast<bf16 *>(attn_smem);
-    bf16 *sK = sQ + kMaxWindowTokens * LD;
+    bf16 *sK = reinterpret_cast<bf16 *>(attn_smem);
     bf16 *sV = sK + kMaxWindowTokens * LD;
     const int seg = blockIdx.x, h = blockIdx.y;
     const int s0 = cu[seg], len = cu[seg + 1] - s0;
@@ -244,39 +245,59 @@ __global__ void __launch_bounds__(32 * kAttnWarps) window_attn_kernel(const bf16
     const int nkt = (len + 15) >> 4;
     const int rows = nkt * 16;
     constexpr int CH = HD / 8;
-    // Asynchronous 16-byte copies straight into shared memory, all in flight at
-    // once; rows past the window's end are zero-filled (source size 0).
-    for (int idx = threadIdx.x; idx < 3 * rows * CH; idx += blockDim.x) {
+    // K and V: asynchronous 16-byte copies straight into shared memory, all in
+    // flight at once; rows past the window's end are zero-filled (source size 0).
+    for (int idx = threadIdx.x; idx < 2 * rows * CH; idx += blockDim.x) {
         const int part = idx / (rows * CH);
         const int rem = idx - part * rows * CH;
         const int r = rem / CH, c = rem - (rem / CH) * CH;
-        const bf16 *src = qkv + (size_t)(s0 + (r < len ? r : 0)) * 3 * d + part * d + h * HD + c * 8;
-        bf16 *dst = (part == 0 ? sQ : part == 1 ? sK : sV) + r * LD + c * 8;
+        const bf16 *src =
+            qkv + (size_t)(s0 + (r < len ? r : 0)) * 3 * d + (part + 1) * d + h * HD + c * 8;
+        bf16 *dst = (part == 0 ? sK : sV) + r * LD + c * 8;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
                      "l"(src), "r"(r < len ? 16 : 0)
                      : "memory");
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
+    asm volatile("cp.async.commit_group;" ::: "memory");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    for (int mt = warp; mt < nkt; mt += kAttnWarps) {
+    // Q: a window has at most 128 tokens = 8 tiles of 16 rows, one per warp; each
+    // warp reads its A fragments straight from global memory (rows past the
+    // window's end read row len - 1 and are dropped).
+    constexpr int KS = HD / 16;
+    static_assert(kMaxWindowTokens <= 16 * kAttnWarps, "one query tile per warp");
+    const int mt = warp;
+    uint32_t qa[KS][4];
+    if (mt < nkt) {
+        const int r0 = min(mt * 16 + g, len - 1), r1 = min(mt * 16 + g + 8, len - 1);
+        const bf16 *q0 = qkv + (size_t)(s0 + r0) * 3 * d + h * HD + 2 * t;
+        const bf16 *q1 = qkv + (size_t)(s0 + r1) * 3 * d + h * HD + 2 * t;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            qa[kk][0] = __ldg(reinterpret_cast<const unsigned int *>(q0 + kk * 16));
+            qa[kk][1] = __ldg(reinterpret_cast<const unsigned int *>(q1 + kk * 16));
+            qa[kk][2] = __ldg(reinterpret_cast<const unsigned int *>(q0 + kk * 16 + 8));
+            qa[kk][3] = __ldg(reinterpret_cast<const unsigned int *>(q1 + kk * 16 + 8));
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+
+    if (mt < nkt) {
         float s[16][4];
 #pragma unroll
         for (int j = 0; j < 16; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-            uint32_t a[4];
-            ldmatrix_x4(a, sQ + (mt * 16 + (lane & 15)) * LD + kk * 16 + (lane >> 4) * 8);
+        for (int kk = 0; kk < KS; ++kk) {
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 if (nt < nkt) {
                     uint32_t b[4];
                     ldmatrix_x4(b, sK + (nt * 16 + (lane & 7) + ((lane >> 4) << 3)) * LD + kk * 16 +
                                        ((lane >> 3) & 1) * 8);
-                    mma_16816(s[2 * nt], a, b[0], b[1]);
-                    mma_16816(s[2 * nt + 1], a, b[2], b[3]);
+                    mma_16816(s[2 * nt], qa[kk], b[0], b[1]);
+                    mma_16816(s[2 * nt + 1], qa[kk], b[2], b[3]);
                 }
             }
         }
@@ -444,23 +465,40 @@ cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, i
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
                              float eps, cudaStream_t st, bool split) {
     if (T <= 0) return cudaSuccess;
-    const int vpl = (d / 4 + 31) / 32;
-    const dim3 grid((T + 7) / 8);
+    const int vpl = (d / 4 + 31) / 32;  // float4 per lane, exact so the row stays in registers
+    const dim3 grid((T + kLnRowsPerBlock - 1) / kLnRowsPerBlock), block(32 * kLnRowsPerBlock);
     const bf16 *gg = static_cast<const bf16 *>(g), *bb = static_cast<const bf16 *>(b);
     bf16 *yy = static_cast<bf16 *>(y);
-    if (vpl <= 4)
-        layernorm_kernel<4><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps, split);
-    else if (vpl <= 8)
-        layernorm_kernel<8><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps, split);
-    else
-        layernorm_kernel<16><<<grid, 256, 0, st>>>(x, gg, bb, yy, T, d, eps, split);
+    const int sp = split ? 1 : 0;
+#define AUT_LN_CASE(V) \
+    case V: layernorm_kernel<V><<<grid, block, 0, st>>>(x, gg, bb, yy, T, d, eps, sp); break;
+    switch (vpl) {
+        AUT_LN_CASE(1)
+        AUT_LN_CASE(2)
+        AUT_LN_CASE(3)
+        AUT_LN_CASE(4)
+        AUT_LN_CASE(5)
+        AUT_LN_CASE(6)
+        AUT_LN_CASE(7)
+        AUT_LN_CASE(8)
+        AUT_LN_CASE(10)
+        AUT_LN_CASE(12)
+        AUT_LN_CASE(16)
+        default:
+            if (vpl <= 12) {
+                layernorm_kernel<12><<<grid, block, 0, st>>>(x, gg, bb, yy, T, d, eps, sp);
+            } else {
+                layernorm_kernel<16><<<grid, block, 0, st>>>(x, gg, bb, yy, T, d, eps, sp);
+            }
+    }
+#undef AUT_LN_CASE
     return cudaGetLastError();
 }
 
 template <int HD>
 cudaError_t run_window_attention(const bf16 *q, bf16 *o, const int *cu_dev, int n_windows, int d,
                                  int heads, float scale_log2e, cudaStream_t st) {
-    constexpr int smem = 3 * kMaxWindowTokens * (HD + 8) * (int)sizeof(bf16);
+    constexpr int smem = 2 * kMaxWindowTokens * (HD + 8) * (int)sizeof(bf16);
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
