@@ -70,21 +70,8 @@ GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &arg
     }
     const int tiles = args.num_m_tiles * args.num_n_tiles;
     const int groups = std::min(tiles, sm_count() / CG);
-    cudaLaunchConfig_t lc{};
-    lc.gridDim = dim3(groups * CG);
-    lc.blockDim = dim3(kGemmThreads);
-    lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
-    lc.stream = st;
-    cudaLaunchAttribute attr[1];
-    if (CG == 2) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        lc.attrs = attr;
-        lc.numAttrs = 1;
-    }
-    const cudaError_t e = cudaLaunchKernelEx(&lc, gemm_tc_kernel<BN, CG>, ta, tb, args);
+    const cudaError_t e = launch_pdl(gemm_tc_kernel<BN, CG>, dim3(groups * CG), dim3(kGemmThreads),
+                                     Cfg::SMEM_BYTES, st, CG, ta, tb, args);
     return e == cudaSuccess ? GemmStatus::kOk : GemmStatus::kLaunch;
 }
 

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;  // 0 issues the MMAs
     const int group = blockIdx.x / CG, n_groups = gridDim.x / CG;
@@ -182,6 +183,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     else
         __syncthreads();
     tc_fence_after();
+    pdl_wait();  // the previous kernel's outputs (this GEMM's A, residual) are complete
     const uint32_t tmem_base = *tmem_slot;
     volatile int *abort_v = abort_flag;
     const int total_tiles = args.num_m_tiles * args.num_n_tiles;

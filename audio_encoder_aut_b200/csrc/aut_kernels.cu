@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
                                                     const bf16 *__restrict__ b,
                                                     bf16 *__restrict__ planes, int plane_rows,
                                                     int C) {
+    pdl_trigger();
+    pdl_wait();
     const int cl = blockIdx.x, hg = blockIdx.y;
     const int4 ci = chunks[chunk_base + cl];
     __shared__ float xs[17][101];  // mel rows 16 hg - 1 .. 16 hg + 15, frames -1 .. 99
@@ -94,6 +96,8 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
 // Zero row, zero column and (odd-column planes) the missing last column of
 // conv3's input planes: the conv2 epilogue never writes them.
 __global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int plane_rows, int C) {
+    pdl_trigger();
+    pdl_wait();
     const int cl = blockIdx.x, plane = blockIdx.y;
     const int CP = C >> 1;
     const size_t row0 = (size_t)plane * plane_rows + (size_t)cl * kP2Rows;
@@ -131,6 +135,8 @@ __global__ void __launch_bounds__(32 * kLnRowsPerBlock) layernorm_kernel(const f
                                                         const bf16 *__restrict__ bt,
                                                         bf16 *__restrict__ y, int T, int d,
                                                         float eps, int split) {
+    pdl_trigger();
+    pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * kLnRowsPerBlock + warp;
     if (row >= T) return;
@@ -239,6 +245,8 @@ __global__ void __launch_bounds__(32 * kAttnWarps) window_attn_kernel(const bf16
     extern __shared__ __align__(16) uint8_t attn_smem[];
     bf16 *sK = reinterpret_cast<bf16 *>(attn_smem);
     bf16 *sV = sK + kMaxWindowTokens * LD;
+    pdl_trigger();
+    pdl_wait();
     const int seg = blockIdx.x, h = blockIdx.y;
     const int s0 = cu[seg], len = cu[seg + 1] - s0;
     if (len <= 0) return;
@@ -439,6 +447,8 @@ __global__ void position_table_kernel(float *pos, int d) {
 // memory: plan tables reach the device without a host buffer that has to
 // outlive the call.
 __global__ void upload_words_kernel(const UploadPayload p, int32_t *dst) {
+    pdl_trigger();
+    pdl_wait();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.n; i += gridDim.x * blockDim.x)
         dst[p.offset + i] = p.words[i];
 }
@@ -448,18 +458,17 @@ cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int c
                          int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
                          int C, cudaStream_t st) {
     if (n_chunks <= 0) return cudaSuccess;
-    conv1_kernel<<<dim3(n_chunks, kC1Rows / 8), 256, 0, st>>>(
-        static_cast<const bf16 *>(feats), T_max, chunks, chunk_base, static_cast<const bf16 *>(w),
-        static_cast<const bf16 *>(b), static_cast<bf16 *>(planes), plane_rows, C);
-    return cudaGetLastError();
+    return launch_pdl(conv1_kernel, dim3(n_chunks, kC1Rows / 8), dim3(256), 0, st, 1,
+                      static_cast<const bf16 *>(feats), T_max, chunks, chunk_base,
+                      static_cast<const bf16 *>(w), static_cast<const bf16 *>(b),
+                      static_cast<bf16 *>(planes), plane_rows, C);
 }
 
 cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int C,
                                    cudaStream_t st) {
     if (n_chunks <= 0) return cudaSuccess;
-    zero_plane_pads_kernel<<<dim3(n_chunks, 4), 256, 0, st>>>(static_cast<bf16 *>(planes),
-                                                             plane_rows, C);
-    return cudaGetLastError();
+    return launch_pdl(zero_plane_pads_kernel, dim3(n_chunks, 4), dim3(256), 0, st, 1,
+                      static_cast<bf16 *>(planes), plane_rows, C);
 }
 
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
@@ -470,8 +479,9 @@ cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void 
     const bf16 *gg = static_cast<const bf16 *>(g), *bb = static_cast<const bf16 *>(b);
     bf16 *yy = static_cast<bf16 *>(y);
     const int sp = split ? 1 : 0;
-#define AUT_LN_CASE(V) \
-    case V: layernorm_kernel<V><<<grid, block, 0, st>>>(x, gg, bb, yy, T, d, eps, sp); break;
+#define AUT_LN_CASE(V)                                                                         \
+    case V:                                                                                    \
+        return launch_pdl(layernorm_kernel<V>, grid, block, 0, st, 1, x, gg, bb, yy, T, d, eps, sp);
     switch (vpl) {
         AUT_LN_CASE(1)
         AUT_LN_CASE(2)
@@ -485,14 +495,13 @@ cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void 
         AUT_LN_CASE(12)
         AUT_LN_CASE(16)
         default:
-            if (vpl <= 12) {
-                layernorm_kernel<12><<<grid, block, 0, st>>>(x, gg, bb, yy, T, d, eps, sp);
-            } else {
-                layernorm_kernel<16><<<grid, block, 0, st>>>(x, gg, bb, yy, T, d, eps, sp);
-            }
+            if (vpl <= 12)
+                return launch_pdl(layernorm_kernel<12>, grid, block, 0, st, 1, x, gg, bb, yy, T, d,
+                                  eps, sp);
+            return launch_pdl(layernorm_kernel<16>, grid, block, 0, st, 1, x, gg, bb, yy, T, d, eps,
+                              sp);
     }
 #undef AUT_LN_CASE
-    return cudaGetLastError();
 }
 
 template <int HD>
@@ -508,9 +517,8 @@ cudaError_t run_window_attention(const bf16 *q, bf16 *o, const int *cu_dev, int 
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    window_attn_kernel<HD><<<dim3(n_windows, heads), 32 * kAttnWarps, smem, st>>>(q, o, cu_dev, d,
-                                                                                  scale_log2e);
-    return cudaGetLastError();
+    return launch_pdl(window_attn_kernel<HD>, dim3(n_windows, heads), dim3(32 * kAttnWarps), smem, st,
+                      1, q, o, cu_dev, d, scale_log2e);
 }
 
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
@@ -567,8 +575,8 @@ cudaError_t launch_upload(const int32_t *host_words, size_t n, int32_t *dst, cud
         p.n = (int)std::min<size_t>(UploadPayload::kWords, n - off);
         p.offset = (int)off;
         std::copy(host_words + off, host_words + off + p.n, p.words);
-        upload_words_kernel<<<(p.n + 255) / 256, 256, 0, st>>>(p, dst);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(upload_words_kernel, dim3((p.n + 255) / 256), dim3(256), 0, st, 1,
+                                   p, dst);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -6,8 +6,37 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 namespace aut {
+
+// Launches a forward-path kernel that may start while the previous kernel in
+// the stream finishes (programmatic dependent launch); the kernel itself waits
+// before touching global memory.  cluster_x > 1 launches CTA clusters.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, int cluster_x, Args &&...args) {
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    lc.attrs = attr;
+    lc.numAttrs = n;
+    return cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+}
 
 enum GemmEpilogue : int {
     kEpiBf16 = 0,        // out bf16 [M, ldo] = acc + bias

@@ -175,6 +175,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
 // erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z),
 // z >= 0, |error| <= 1.5e-7; odd symmetry for z < 0.
+// Programmatic dependent launch: let the next kernel in the stream start its
+// launch and set-up now; and wait until the previous kernel has completed and
+// its memory is visible.  Every kernel of the forward waits before its first
+// global-memory access, so stream order is kept for all data.
+AUT_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+AUT_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 AUT_DEV float gelu_fast(float x) {
     const float z = fabsf(x) * 0.70710678118654752f;
     const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));

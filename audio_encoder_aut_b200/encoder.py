@@ -126,6 +126,30 @@ class Encoder:
             raise A.AutError(st, "aut_encode_packed")
         return out
 
+    def capture(self, features: torch.Tensor, feature_lens, out: torch.Tensor | None = None,
+                warmup: int = 2):
+        """Records one aut_encode of this exact batch shape into a CUDA graph and
+        returns (graph, out).  The plan is built on the host once, outside the
+        graph (aut_encoder page, module docstring: the runner's plan is built
+        outside the graph so the block loop replays as a CUDA graph); replaying
+        the graph re-runs the whole forward on whatever `features` then holds.
+        The graph keeps this encoder's workspace, so it must not be replayed
+        concurrently with another call on the same encoder."""
+        if out is None:
+            _, _, total, _, _ = self.plan(feature_lens)
+            out = torch.empty((total, self.cfg.output_dim), dtype=torch.float32, device=self.device)
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            for _ in range(warmup):  # one-time kernel attributes, workspace sizing
+                self.encode(features, feature_lens, out=out)
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        torch.cuda.synchronize(self.device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self.encode(features, feature_lens, out=out)
+        return graph, out
+
     def check(self) -> int:
         """Device status of the latest call on this encoder's workspace."""
         return A.aut_check(self._ws.data_ptr()) if self._ws is not None else A.AUT_OK

@@ -216,13 +216,18 @@ def our_arm(args, rank, world, local_rank):
         barrier()
         return [a.elapsed_time(b) for a, b in evs]
 
+    if args.graph:
+        graph, _ = enc.capture(fd, lens, out=out)
+        step = graph.replay
+    else:
+        step = lambda: enc.encode(fd, lens, out=out)  # noqa: E731
     for _ in range(args.warmup):
-        enc.encode(fd, lens, out=out)
+        step()
     torch.cuda.synchronize()
     assert enc.check() == A.AUT_OK
 
     sampler = ClockSampler(dev)
-    step_ms = timed(lambda: enc.encode(fd, lens, out=out), args.steps)
+    step_ms = timed(step, args.steps)
     clocks = sampler.stop()
     status = enc.check()
     total_ms = sum(step_ms)
@@ -272,7 +277,7 @@ def our_arm(args, rank, world, local_rank):
 
     def e2e_step():
         fd.copy_(h_feats, non_blocking=True)
-        enc.encode(fd, lens, out=out)
+        step()
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(2):
@@ -308,6 +313,7 @@ def our_arm(args, rank, world, local_rank):
                        "audio_seconds": audio_s, "total_tokens": T, "windows": nW,
                        "chunks": nch, "d_model": cfg.d_model, "layers": cfg.encoder_layers,
                        "l2": "256 MiB buffer written between timed steps (outside the events)",
+                       "launch": "CUDA graph of the whole forward" if args.graph else "eager",
                        "parallelism": f"dp{world} (weak: one batch per GPU)"},
             "tokens_per_s": tokens_s,
             "tflops": flops / (ms / 1e3) / 1e12,
@@ -341,6 +347,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="omni_16req", choices=sorted(S.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch the forward eagerly instead of replaying its CUDA graph")
     ap.add_argument("--cpu-sample-seconds", type=float, default=60.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

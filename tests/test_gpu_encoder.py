@@ -198,3 +198,22 @@ def test_stem_group_boundaries():
     out = run(enc, feats, lens)
     ref, _ = O.forward(cfg, w, feats, lens)
     assert_rows_close(out, ref, "grouped stem")
+
+
+def test_cuda_graph_replay_matches_eager_bit_exact():
+    """The forward captured once into a CUDA graph (plan built on the host,
+    outside the graph) and replayed on new features gives the eager result."""
+    cfg, w, enc = encoder("omni_16req")
+    lens = [777, 1203, 64]
+    fa, fb = S.features(lens, seed=11), S.features(lens, seed=12)
+    feats_dev = enc.features_to_device(fa)
+    graph, out = enc.capture(feats_dev, lens)
+    feats_dev.copy_(enc.features_to_device(fb))
+    graph.replay()
+    torch.cuda.synchronize()
+    assert enc.check() == A.AUT_OK
+    got = out.cpu().numpy().copy()
+    eager = run(enc, fb, lens)
+    assert np.array_equal(got, eager)
+    ref, _ = O.forward(cfg, w, fb, lens, dtype=np.float32)
+    assert_rows_close(got, ref, "graph replay")
