@@ -271,13 +271,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // -------------------------------------------------- MMA issuer --
             constexpr uint32_t idesc = idesc_bf16_f32(128 * CG, BN);
             constexpr uint16_t kPair = 0x3;
+            const bool resid_mode = args.epi == kEpiResidF32;
             int stage = 0, it = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = group; ok && tile < total_tiles; tile += n_groups, ++it) {
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
-                if (!mbar_wait(tempty + acc, acc_phase ^ 1u, abort_v, lim)) {
+                // Residual mode: wait for the accumulator's preload (phase = use
+                // index); otherwise for the epilogue to have drained it (the phase
+                // before the first use counts as complete).
+                const uint32_t want = resid_mode ? acc_phase : (acc_phase ^ 1u);
+                if (!mbar_wait(tempty + acc, want, abort_v, lim)) {
                     ok = false;
                     break;
                 }
@@ -293,12 +298,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint64_t b_desc = smem_desc_sw128(sB + stage * Cfg::B_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {  // K = 16 per MMA: +32 bytes in the row
+                        const uint32_t accumulate = resid_mode || (kb | kk) != 0;
                         if constexpr (CG == 2)
                             tc_mma_bf16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
-                                             (kb | kk) != 0);
+                                             accumulate);
                         else
                             tc_mma_bf16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
-                                        (kb | kk) != 0);
+                                        accumulate);
                     }
                     if constexpr (CG == 2)
                         tc_commit_pair(empty + stage, kPair);
@@ -325,31 +331,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ------------------------------------------------------- epilogue --
-        // Eight warps: TMEM lane quadrant (warp % 4) x column half (alternate
-        // 16-column chunks).  Two chunks are loaded per TMEM wait, and the
-        // residual rows they update are fetched before that wait.
+        // Eight warps: TMEM lane quadrant (warp % 4) x column parity (alternate
+        // 16-column chunks); two chunks per TMEM wait.
+        // Residual mode: the accumulator is pre-loaded with x + bias (tcgen05.st)
+        // while the MMAs run on the other accumulator, the MMAs add onto it, and
+        // draining is a plain store - no load sits on the tile's critical path.
         const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
         const int half = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
         constexpr int NC = BN / 16;
-        int it = 0;
+        const bool resid = args.epi == kEpiResidF32;
         bool ok = true;
         const uint32_t tempty_even = CG == 2 ? map_to_rank(tempty, 0) : 0;
-        for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
-            if (!mbar_wait(tfull + acc, acc_phase, abort_v, lim)) {
-                ok = false;
-                break;
+        auto release = [&](int acc) {  // accumulator `acc` may be (re)written by the MMAs
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (CG == 2)
+                    mbar_arrive_cluster(tempty_even + acc * 8);
+                else
+                    mbar_arrive(tempty + acc);
             }
-            tc_fence_after();
-            const int n_blk = tile % args.num_n_tiles;
+        };
+        // Where this thread's accumulator row of `tile` goes.
+        auto locate = [&](int tile, bool &valid, size_t &dst_row, int &pos_row) {
             const int m_blk = (tile / args.num_n_tiles) * CG + (int)rank;  // 128-row slot
-
-            // Where this thread's accumulator row goes.
-            bool valid = true;
-            size_t dst_row = 0;  // element offset of column 0 of the row
-            int pos_row = 0;
+            valid = true;
+            dst_row = 0;
+            pos_row = 0;
             if (args.conv) {
                 const int vr_local = r / args.conv_cols;
                 const int j = r - vr_local * args.conv_cols;
@@ -359,8 +368,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 valid = vr_local < args.conv_rows && i < args.conv_vrows - 1 &&
                         chunk < args.conv_chunks;
                 if (args.epi == kEpiConvPlanes) {
-                    // conv2 output (row i, col j) -> phase plane ((i&1), (j&1)) of conv3's input,
-                    // behind one zero row and one zero column.
+                    // conv2 output (row i, col j) -> phase plane ((i&1), (j&1)) of conv3's
+                    // input, behind one zero row and one zero column.
                     const int plane = (i & 1) * 2 + (j & 1);
                     const size_t prow = (size_t)plane * args.dst_plane_rows +
                                         (size_t)chunk * args.dst_chunk_rows + (i >> 1) + 1;
@@ -386,7 +395,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     dst_row = (size_t)m * args.ldo;
                 }
             }
+        };
+        // Residual mode: accumulator `acc` <- x + bias over this thread's row and chunks.
+        auto preload = [&](int tile, int acc) {
+            bool valid;
+            size_t dst_row;
+            int pos_row;
+            locate(tile, valid, dst_row, pos_row);
+            const int n_base = (tile % args.num_n_tiles) * BN;
+            const float *xp = reinterpret_cast<const float *>(args.out) + dst_row + n_base;
+            const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+#pragma unroll 1
+            for (int c0 = half; c0 < NC; c0 += 8) {  // four chunks of loads in flight
+                float v[4][16];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + 2 * u;
+                    if (c < NC) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 e = valid ? reinterpret_cast<const float4 *>(xp + c * 16)[q]
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                            v[u][4 * q] = e.x;
+                            v[u][4 * q + 1] = e.y;
+                            v[u][4 * q + 2] = e.z;
+                            v[u][4 * q + 3] = e.w;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + 2 * u;
+                    if (c < NC) {
+                        add_bias16(v[u], args.bias, n_base + c * 16);
+                        tmem_st16(t_addr + c * 16, v[u]);
+                    }
+                }
+            }
+            tc_wait_st();
+            release(acc);
+        };
 
+        if (resid) {  // the first two accumulators start from the residual
+            int t = group;
+            for (int a = 0; a < 2 && t < total_tiles; ++a, t += n_groups) preload(t, a);
+        }
+        int it = 0;
+        for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(tfull + acc, acc_phase, abort_v, lim)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int n_blk = tile % args.num_n_tiles;
+            bool valid;
+            size_t dst_row;
+            int pos_row;
+            locate(tile, valid, dst_row, pos_row);
             const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
             for (int c0 = half; c0 < NC; c0 += 4) {
@@ -395,56 +462,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 float v0[16], v1[16];
                 tmem_ld16(t_addr + c0 * 16, v0);
                 if (two) tmem_ld16(t_addr + c1 * 16, v1);
-                float4 res0[4], res1[4];
-                float *rp = reinterpret_cast<float *>(args.out) + dst_row;
-                if (args.epi == kEpiResidF32 && valid) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) res0[q] = reinterpret_cast<const float4 *>(rp + c0 * 16 + n_blk * BN)[q];
-                    if (two)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) res1[q] = reinterpret_cast<const float4 *>(rp + c1 * 16 + n_blk * BN)[q];
-                }
                 tc_wait_ld();
                 if (!valid) continue;
+                float *rp = reinterpret_cast<float *>(args.out) + dst_row;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     if (k == 1 && !two) break;
                     float(&v)[16] = k ? v1 : v0;
-                    const float4(&res)[4] = k ? res1 : res0;
                     const int n0 = n_blk * BN + (k ? c1 : c0) * 16;
-                    add_bias16(v, args.bias, n0);
+                    if (!resid) add_bias16(v, args.bias, n0);
                     switch (args.epi) {
                         case kEpiBf16:
                             store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
                             break;
                         case kEpiBf16Gelu:
                         case kEpiConvPlanes:
-                        case kEpiConvFlat:
+                        case kEpiConvFlat: {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) v[i] = gelu_fast(v[i]);
+                            for (int i = 0; i < 16; i += 2) {
+                                const float2 g = gelu_fast2(make_float2(v[i], v[i + 1]));
+                                v[i] = g.x;
+                                v[i + 1] = g.y;
+                            }
                             store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
                             break;
+                        }
                         case kEpiBf16GeluSplit: {
                             // GELU, then the value as hi + lo bf16 halves [hi | lo] of a 2N row.
                             float lo[16];
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                v[i] = gelu_fast(v[i]);
-                                lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
+                            for (int i = 0; i < 16; i += 2) {
+                                const float2 g = gelu_fast2(make_float2(v[i], v[i + 1]));
+                                v[i] = g.x;
+                                v[i + 1] = g.y;
                             }
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
                             __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0;
                             store_bf16x16(o, v);
                             store_bf16x16(o + args.N, lo);
                             break;
                         }
-                        case kEpiResidF32: {
-                            float4 *p = reinterpret_cast<float4 *>(rp + n0);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                p[q] = make_float4(res[q].x + v[4 * q], res[q].y + v[4 * q + 1],
-                                                   res[q].z + v[4 * q + 2], res[q].w + v[4 * q + 3]);
-                            break;
-                        }
+                        case kEpiResidF32:  // accumulator already holds x + bias + X W^T
                         case kEpiF32:
                         case kEpiPackTokens: {
                             if (args.epi == kEpiPackTokens && args.pos) {
@@ -470,13 +530,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if constexpr (CG == 2)
-                    mbar_arrive_cluster(tempty_even + acc * 8);
-                else
-                    mbar_arrive(tempty + acc);
+            if (resid) {
+                const int next = tile + 2 * n_groups;  // the tile this accumulator serves next
+                if (next < total_tiles) {
+                    tc_fence_before();  // finish reading the drained values before rewriting
+                    preload(next, acc);
+                }
+            } else {
+                release(acc);
             }
         }
         if (!ok && lane == 0) gemm_signal_abort(args, abort_v);

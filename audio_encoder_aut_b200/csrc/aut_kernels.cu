@@ -22,8 +22,9 @@ using bf16 = __nv_bfloat16;
 // output (h, w) at (h/2 + 1, w/2 + 1).  conv2's filter tap (kh, kw) then reads
 // one plane at a fixed offset, a plain rectangle a TMA box can fetch.
 //
-// Block (chunk, 8 output rows); each thread computes four channels for a
-// strided set of positions, so a warp writes 32 consecutive channel quads.
+// Block (chunk, 8 output rows); each thread computes eight channels (packed
+// fp32x2 arithmetic) for a strided set of positions, so a warp writes 32
+// consecutive 16-byte channel octets.
 __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ feats, int T_max,
                                                     const int4 *__restrict__ chunks,
                                                     int chunk_base, const bf16 *__restrict__ w,
@@ -36,60 +37,76 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
     const int4 ci = chunks[chunk_base + cl];
     __shared__ float xs[17][101];  // mel rows 16 hg - 1 .. 16 hg + 15, frames -1 .. 99
     const bf16 *src = feats + ((size_t)ci.x * kMelBins) * T_max + ci.y;
-    for (int idx = threadIdx.x; idx < 17 * 101; idx += blockDim.x) {
+    // All of this thread's loads are issued before any is used (one round trip).
+    constexpr int kTile = 17 * 101, kPer = (kTile + 255) / 256;
+    float vals[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int idx = threadIdx.x + u * blockDim.x;
         const int rr = idx / 101, cc = idx - rr * 101;
         const int mel = 16 * hg - 1 + rr, fr = cc - 1;
-        float v = 0.f;
-        if (mel >= 0 && mel < kMelBins && fr >= 0 && fr < ci.z)
-            v = __bfloat162float(src[(size_t)mel * T_max + fr]);
-        xs[rr][cc] = v;
+        vals[u] = (idx < kTile && mel >= 0 && mel < kMelBins && fr >= 0 && fr < ci.z)
+                      ? __bfloat162float(src[(size_t)mel * T_max + fr])
+                      : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int idx = threadIdx.x + u * blockDim.x;
+        if (idx < kTile) (&xs[0][0])[idx] = vals[u];
     }
     __syncthreads();
 
-    const int CQ = C >> 2;  // channel quads
-    const int slices = blockDim.x / CQ;
-    const int cq = threadIdx.x % CQ, slice = threadIdx.x / CQ;
+    const int CO = C >> 3;  // channel octets
+    const int slices = blockDim.x / CO;
+    const int co = threadIdx.x % CO, slice = threadIdx.x / CO;
     if (slice >= slices) return;
-    float wt[4][9], bias[4];
+    float2 wt[4][9], bias[4];  // channel pairs (2p, 2p + 1) of this thread's octet
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int p = 0; p < 4; ++p) {
+        const int c = 8 * co + 2 * p;
 #pragma unroll
-        for (int k = 0; k < 9; ++k) wt[c][k] = __bfloat162float(w[(4 * cq + c) * 9 + k]);
-        bias[c] = __bfloat162float(b[4 * cq + c]);
+        for (int k = 0; k < 9; ++k)
+            wt[p][k] = make_float2(__bfloat162float(w[c * 9 + k]), __bfloat162float(w[(c + 1) * 9 + k]));
+        bias[p] = make_float2(__bfloat162float(b[c]), __bfloat162float(b[c + 1]));
     }
     const size_t chunk_row0 = (size_t)cl * kP1Rows;
     for (int pos = slice; pos < 8 * kC1Cols; pos += slices) {
         const int hl = pos / kC1Cols, wo = pos - hl * kC1Cols;
-        float x[9];
+        float2 x[9];
 #pragma unroll
         for (int kh = 0; kh < 3; ++kh)
 #pragma unroll
-            for (int kw = 0; kw < 3; ++kw) x[kh * 3 + kw] = xs[2 * hl + kh][2 * wo + kw];
-        float a[4];
+            for (int kw = 0; kw < 3; ++kw) {
+                const float v = xs[2 * hl + kh][2 * wo + kw];
+                x[kh * 3 + kw] = make_float2(v, v);
+            }
+        uint32_t packed[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            a[c] = bias[c];
+        for (int p = 0; p < 4; ++p) {
+            float2 a = bias[p];
 #pragma unroll
-            for (int k = 0; k < 9; ++k) a[c] = fmaf(wt[c][k], x[k], a[c]);
+            for (int k = 0; k < 9; ++k) a = ffma2(wt[p][k], x[k], a);
+            const float2 g = gelu_fast2(a);
+            packed[p] = pack_bf16x2(g.x, g.y);
         }
         const int h = 8 * hg + hl;
         const int plane = (h & 1) * 2 + (wo & 1);
         const size_t row = (size_t)plane * plane_rows + chunk_row0 + (h >> 1) + 1;
-        uint2 *dst = reinterpret_cast<uint2 *>(planes + (row * kP1Cols + (wo >> 1) + 1) * C) + cq;
-        *dst = make_uint2(pack_bf16x2(gelu_fast(a[0]), gelu_fast(a[1])),
-                          pack_bf16x2(gelu_fast(a[2]), gelu_fast(a[3])));
+        uint4 *dst = reinterpret_cast<uint4 *>(planes + (row * kP1Cols + (wo >> 1) + 1) * C) + co;
+        *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
     // Zero column of the plane rows this block owns, and (first block) the zero row.
     for (int idx = slice; idx < 16; idx += slices) {
         const int plane = idx >> 2, r = 4 * hg + (idx & 3) + 1;
         const size_t row = (size_t)plane * plane_rows + chunk_row0 + r;
-        reinterpret_cast<uint2 *>(planes + row * kP1Cols * C)[cq] = make_uint2(0u, 0u);
+        reinterpret_cast<uint4 *>(planes + row * kP1Cols * C)[co] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (hg == 0)
         for (int idx = slice; idx < 4 * kP1Cols; idx += slices) {
             const int plane = idx / kP1Cols, col = idx - plane * kP1Cols;
             const size_t row = (size_t)plane * plane_rows + chunk_row0;
-            reinterpret_cast<uint2 *>(planes + (row * kP1Cols + col) * C)[cq] = make_uint2(0u, 0u);
+            reinterpret_cast<uint4 *>(planes + (row * kP1Cols + col) * C)[co] =
+                make_uint4(0u, 0u, 0u, 0u);
         }
 }
 
@@ -127,7 +144,7 @@ __global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int 
 // two passes (mean, then centred variance).  With `split`, the output row is
 // [hi | lo] (2 d wide): hi = bf16(y), lo = bf16(y - hi), so that a GEMM over
 // the doubled K against [W | W] sees y to about 16 significant bits.
-constexpr int kLnRowsPerBlock = 4;  // one warp per row
+constexpr int kLnRowsPerBlock = 8;  // one warp per row
 
 template <int VPL>  // float4 per lane
 __global__ void __launch_bounds__(32 * kLnRowsPerBlock) layernorm_kernel(const float *__restrict__ x,
@@ -144,15 +161,6 @@ __global__ void __launch_bounds__(32 * kLnRowsPerBlock) layernorm_kernel(const f
     const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)row * d);
     const uint2 *gr = reinterpret_cast<const uint2 *>(g);
     const uint2 *br = reinterpret_cast<const uint2 *>(bt);
-    uint2 gg[VPL], bb[VPL];
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {  // gamma/beta in flight while the row is reduced
-        const int idx = lane + 32 * i;
-        if (idx < n4) {
-            gg[i] = __ldg(gr + idx);
-            bb[i] = __ldg(br + idx);
-        }
-    }
     float4 v[VPL];
     float s = 0.f;
 #pragma unroll
@@ -183,10 +191,11 @@ __global__ void __launch_bounds__(32 * kLnRowsPerBlock) layernorm_kernel(const f
     for (int i = 0; i < VPL; ++i) {
         const int idx = lane + 32 * i;
         if (idx < n4) {
-            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg[i].x));
-            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg[i].y));
-            const float2 c0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb[i].x));
-            const float2 c1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb[i].y));
+            const uint2 gg = __ldg(gr + idx), bb = __ldg(br + idx);  // same for every row: L1 hits
+            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg.x));
+            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gg.y));
+            const float2 c0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb.x));
+            const float2 c1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bb.y));
             const float o0 = (v[i].x - mean) * rstd * g0.x + c0.x;
             const float o1 = (v[i].y - mean) * rstd * g0.y + c0.y;
             const float o2 = (v[i].z - mean) * rstd * g1.x + c1.x;

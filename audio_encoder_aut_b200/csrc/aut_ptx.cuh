@@ -151,6 +151,22 @@ AUT_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+AUT_DEV void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Stores 16 consecutive fp32 columns into this thread's TMEM lane.
+AUT_DEV void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
 // with 128-byte swizzling: rows of 128 bytes (64 bf16 of K), 8-row swizzle
 // atoms 1024 bytes apart.  Fields: start address >> 4 (bits 0-13), leading
@@ -171,10 +187,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            ((uint32_t)(M >> 4) << 24);
 }
 
-// GELU(x) = x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2 (the exact form), with erf
-// from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
-// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z),
-// z >= 0, |error| <= 1.5e-7; odd symmetry for z < 0.
 // Programmatic dependent launch: let the next kernel in the stream start its
 // launch and set-up now; and wait until the previous kernel has completed and
 // its memory is visible.  Every kernel of the forward waits before its first
@@ -182,16 +194,49 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 AUT_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 AUT_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// GELU(x) = x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2 (the exact form), with erf
+// from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.25:
+// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3) exp(-z^2), t = 1 / (1 + p z), z >= 0,
+// |error| <= 2.5e-5 (two orders below the bf16 rounding of the results);
+// odd symmetry for z < 0.
+constexpr float kErfP = 0.47047f, kErfA1 = 0.3480242f, kErfA2 = -0.0958798f,
+                kErfA3 = 0.7478556f;
+
 AUT_DEV float gelu_fast(float x) {
     const float z = fabsf(x) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
-    float p = fmaf(1.061405429f, t, -1.453152027f);
-    p = fmaf(p, t, 1.421413741f);
-    p = fmaf(p, t, -0.284496736f);
-    p = fmaf(p, t, 0.254829592f);
-    p *= t;
-    const float erf_abs = fmaf(-p, __expf(-z * z), 1.0f);
+    const float t = __fdividef(1.0f, fmaf(kErfP, z, 1.0f));
+    const float poly = fmaf(fmaf(kErfA3, t, kErfA2), t, kErfA1) * t;
+    const float erf_abs = fmaf(-poly, __expf(-z * z), 1.0f);
     return 0.5f * x * (1.0f + copysignf(erf_abs, x));
+}
+
+// Packed fp32x2 arithmetic (two lanes per instruction).
+AUT_DEV unsigned long long f2_bits(float2 v) { return *reinterpret_cast<unsigned long long *>(&v); }
+AUT_DEV float2 f2_from(unsigned long long b) { return *reinterpret_cast<float2 *>(&b); }
+AUT_DEV float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+    return f2_from(d);
+}
+AUT_DEV float2 fmul2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return f2_from(d);
+}
+
+// gelu_fast on two values, the polynomial and scaling in packed fp32x2.
+AUT_DEV float2 gelu_fast2(float2 x) {
+    const float2 z = make_float2(fabsf(x.x) * 0.70710678118654752f, fabsf(x.y) * 0.70710678118654752f);
+    const float2 den = ffma2(make_float2(kErfP, kErfP), z, make_float2(1.f, 1.f));
+    const float2 t = make_float2(__fdividef(1.0f, den.x), __fdividef(1.0f, den.y));
+    float2 poly = ffma2(make_float2(kErfA3, kErfA3), t, make_float2(kErfA2, kErfA2));
+    poly = ffma2(poly, t, make_float2(kErfA1, kErfA1));
+    poly = fmul2(poly, t);
+    const float2 zz = fmul2(z, z);
+    const float2 e = make_float2(__expf(-zz.x), __expf(-zz.y));
+    const float2 erf_abs = ffma2(make_float2(-poly.x, -poly.y), e, make_float2(1.f, 1.f));
+    const float2 one_plus = make_float2(1.0f + copysignf(erf_abs.x, x.x), 1.0f + copysignf(erf_abs.y, x.y));
+    return fmul2(fmul2(make_float2(0.5f, 0.5f), x), one_plus);
 }
 
 AUT_DEV uint32_t pack_bf16x2(float a, float b) {
