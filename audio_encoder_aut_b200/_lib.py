@@ -86,6 +86,8 @@ _SIGNATURES = {
                                 c_float, c_void_p]),
     "aut_window_attention": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                        POINTER(c_int32), c_int32, c_void_p, c_size_t, c_void_p]),
+    "aut_window_attention_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32,
+                                               POINTER(c_int32), c_int32, c_void_p]),
     "aut_check": (c_int32, [c_void_p]),
     "aut_check_status_word": (c_int32, [c_void_p]),
     "aut_status_string": (c_char_p, [c_int32]),
@@ -221,6 +223,14 @@ def aut_window_attention(qkv: int, out: int, T: int, d: int, heads: int, cu_seql
                          workspace: int, ws_bytes: int, stream: int) -> int:
     return lib().aut_window_attention(qkv, out, T, d, heads, _i32(cu_seqlens),
                                       len(cu_seqlens) - 1, workspace, ws_bytes, stream)
+
+
+def aut_window_attention_noalloc(qkv: int, out: int, T: int, d: int, heads: int, cu_seqlens,
+                                 stream: int) -> int:
+    """Window attention without a caller workspace (scratch in the library's own
+    device array; see include/aut.h for its limits)."""
+    return lib().aut_window_attention_noalloc(qkv, out, T, d, heads, _i32(cu_seqlens),
+                                              len(cu_seqlens) - 1, stream)
 
 
 def aut_check(workspace: int) -> int:

@@ -231,6 +231,29 @@ aut_status aut_window_attention(const void *qkv, void *out, int32_t T, int32_t d
                                 const int32_t *cu_seqlens, int32_t num_windows,
                                 void *workspace, size_t ws_bytes, aut_stream_t stream);
 
+/* Window attention that allocates nothing, for callers that cannot allocate
+ * device memory: code whose device memory belongs to another allocator that
+ * forbids raw cudaMalloc, or code running where allocation is not allowed
+ * (for example during a CUDA-graph capture that rejects allocation calls).
+ * There is no counterpart in the paper; this computes exactly what
+ * aut_window_attention computes, with the same argument meanings, but keeps
+ * its scratch (the uploaded cu_seqlens) in a file-scope device array of the
+ * library instead of a caller workspace.
+ * Limits and behaviour:
+ *   - num_windows at most 32767 (128 KiB of scratch); larger returns
+ *     AUT_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every GPU that loads the library holds the array until the process
+ *     exits.
+ *   - All calls share the array, which keeps the last call's contents: calls
+ *     that overlap on the GPU (unordered streams) race and must not be issued.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called. */
+aut_status aut_window_attention_noalloc(const void *qkv, void *out, int32_t T, int32_t d,
+                                        int32_t heads, const int32_t *cu_seqlens,
+                                        int32_t num_windows, aut_stream_t stream);
+
 /* Reads and clears the device status word of a workspace used by aut_encode /
  * aut_frontend / aut_encode_packed (synchronous: call after the stream is
  * synchronised).  Each of those calls clears the word when it starts, so this
