@@ -24,7 +24,8 @@ LIB = os.path.join(PKG, "libaut.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
               "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include"), "-I", CSRC]
-SOURCES = ["aut_plan.cpp", "aut_kernels.cu", "aut_gemm.cu", "aut_api.cu", "aut_noalloc.cu"]
+SOURCES = ["aut_plan.cpp", "aut_kernels.cu", "aut_gemm.cu", "aut_attention.cu", "aut_api.cu",
+           "aut_noalloc.cu"]
 
 
 def nvcc() -> str:

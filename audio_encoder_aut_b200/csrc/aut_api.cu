@@ -240,7 +240,8 @@ aut_status run_encode(const Ctx &c, float *x, int T, int nW, int n_layers, void 
         AUT_TRY(cuda_status(launch_layernorm(x, lw.ln1_w, lw.ln1_b, xn, T, d, cfg->ln_eps, c.st)));
         AUT_TRY(c.mark(AUT_K_LAYERNORM));
         AUT_TRY(linear(c, xn, lw.qkv_w, lw.qkv_b, qkv, T, 3 * d, d, kEpiBf16, AUT_K_QKV));
-        AUT_TRY(cuda_status(launch_window_attention(qkv, attn, cu, nW, d, cfg->heads, c.st)));
+        AUT_TRY(cuda_status(launch_window_attention(qkv, attn, cu, nW, d, cfg->heads, c.st, T,
+                                                    c.status)));
         AUT_TRY(c.mark(AUT_K_ATTENTION));
         // attention output [hi | lo] against [o_w | o_w]
         const void *o_w2 = static_cast<const uint8_t *>(c.w->o_w_dup) + (size_t)l * d * 2 * d * 2;
@@ -504,7 +505,7 @@ extern "C" aut_status aut_window_attention(const void *qkv, void *out, int32_t T
     AUT_TRY(cuda_status(launch_upload(cu_seqlens, (size_t)num_windows + 1,
                                       static_cast<int32_t *>(workspace), st)));
     return cuda_status(launch_window_attention(qkv, out, static_cast<const int *>(workspace),
-                                               num_windows, d, heads, st));
+                                               num_windows, d, heads, st, T));
 }
 
 extern "C" aut_status aut_check_status_word(int32_t *status) {

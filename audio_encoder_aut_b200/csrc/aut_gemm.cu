@@ -44,6 +44,22 @@ bool make_map(CUtensorMap *m, int rank, const void *ptr, const cuuint64_t *dims,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
+                                const uint64_t *strides, const uint32_t *box) {
+    cuuint64_t dd[5], ss[4];
+    cuuint32_t bb[5];
+    for (int i = 0; i < rank; ++i) {
+        dd[i] = dims[i];
+        bb[i] = box[i];
+        if (i + 1 < rank) ss[i] = strides[i];
+    }
+    return make_map(m, rank, ptr, dd, ss, bb);
+}
+
+namespace {
+
 int sm_count() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);

@@ -531,9 +531,11 @@ cudaError_t run_window_attention(const bf16 *q, bf16 *o, const int *cu_dev, int 
 }
 
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
-                                    int d, int heads, cudaStream_t st) {
+                                    int d, int heads, cudaStream_t st, int T, int *status) {
     if (n_windows <= 0) return cudaSuccess;
     const int hd = d / heads;
+    if (hd == 64 && T > 0)
+        return launch_window_attention_tc(qkv, out, cu_dev, n_windows, d, heads, T, status, st);
     const float scale_log2e = 1.4426950408889634f / sqrtf((float)hd);
     const bf16 *q = static_cast<const bf16 *>(qkv);
     bf16 *o = static_cast<bf16 *>(out);

@@ -2,6 +2,7 @@
 // aut_gemm.cu), used by the C-ABI layer in aut_api.cu.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -64,7 +65,15 @@ cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void 
                              float eps, cudaStream_t st, bool split = false);
 cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st);
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
-                                    int d, int heads, cudaStream_t st);
+                                    int d, int heads, cudaStream_t st, int T = -1,
+                                    int *status = nullptr);
+// tcgen05 variant for head_dim 64 (aut_attention.cu); T = rows of qkv.
+cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu_dev, int n_windows,
+                                       int d, int heads, int T, int *status, cudaStream_t st);
+// bf16 tensor map with 128-byte swizzle (aut_gemm.cu): dims innermost first,
+// strides in bytes for dims 1.., box in elements.
+bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
+                                const uint64_t *strides, const uint32_t *box);
 cudaError_t launch_prepare(const void *conv2_w, const void *conv3_w, const void *conv_out_w,
                            void *conv2_tap, void *conv3_tap, void *conv_out_fc, float *pos, int C,
                            int d, cudaStream_t st);

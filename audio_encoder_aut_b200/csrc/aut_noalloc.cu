@@ -74,7 +74,7 @@ extern "C" aut_status aut_window_attention_noalloc(const void *qkv, void *out, i
     // needs to start at zero.
     if (launch_upload(cu_seqlens, (size_t)num_windows + 1, scratch, s) != cudaSuccess)
         return AUT_ERR_CUDA;
-    return launch_window_attention(qkv, out, scratch, num_windows, d, heads, s) == cudaSuccess
+    return launch_window_attention(qkv, out, scratch, num_windows, d, heads, s, T) == cudaSuccess
                ? AUT_OK
                : AUT_ERR_CUDA;
 }

@@ -151,6 +151,25 @@ AUT_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Loads 32 consecutive fp32 columns of this thread's TMEM lane.
+AUT_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 AUT_DEV void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Stores 16 consecutive fp32 columns into this thread's TMEM lane.
@@ -177,6 +196,23 @@ AUT_DEV uint64_t smem_desc_sw128(const void *tile) {
     const uint64_t addr = smem_addr(tile);
     return ((addr & 0x3FFFFull) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
            (2ull << 61);
+}
+
+// Descriptor for an MN-major operand tile (the N, or M, index contiguous) with
+// 128-byte swizzling: rows of 128 bytes hold 64 bf16 of N for one K index;
+// groups of 8 K rows (1024-byte swizzle atoms) follow at the stride byte offset
+// 1024 >> 4.  The tile here is exactly 64 wide in N, so the leading byte
+// offset (between 64-wide N groups) is never used.
+AUT_DEV uint64_t smem_desc_sw128_mn(const void *tile) {
+    const uint64_t addr = smem_addr(tile);
+    return ((addr & 0x3FFFFull) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Fence making this thread's generic-proxy shared-memory writes visible to the
+// async proxy (TMA, tcgen05.mma) after a subsequent barrier.
+AUT_DEV void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator,
