@@ -16,7 +16,7 @@ AUT_OK, AUT_ERR_INVALID_ARG, AUT_ERR_UNSUPPORTED, AUT_ERR_WORKSPACE, AUT_ERR_CUD
     AUT_ERR_TIMEOUT = range(6)
 
 EPI_BF16, EPI_BF16_GELU, EPI_RESID_F32, EPI_F32 = 0, 1, 2, 3
-LINEAR_FAULT_INJECT, LINEAR_SINGLE_CTA = 1, 2
+LINEAR_FAULT_INJECT, LINEAR_SINGLE_CTA, LINEAR_F16 = 1, 2, 4
 
 KERNEL_KINDS = ["upload", "zero_pads", "conv1", "conv2", "conv3", "conv_out", "layernorm",
                 "qkv", "attention", "o_proj", "fc1", "fc2", "proj1", "proj2"]
@@ -45,7 +45,7 @@ class aut_weights(ctypes.Structure):
                 + [(n, c_void_p) for n in ["ln_post_w", "ln_post_b", "proj1_w", "proj1_b",
                                            "proj2_w", "proj2_b", "conv2_w_tap", "conv3_w_tap",
                                            "conv_out_w_fc", "pos_table", "proj1_w_dup",
-                                           "proj2_w_dup", "o_w_dup"]])
+                                           "proj2_w_dup", "o_w_f16"]])
 
 
 class aut_trace(ctypes.Structure):

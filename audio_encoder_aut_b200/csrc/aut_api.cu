@@ -36,7 +36,7 @@ struct Region {
 };
 
 struct PreparedLayout {
-    size_t conv2, conv3, conv_out, pos, proj1_dup, proj2_dup, o_dup, total;
+    size_t conv2, conv3, conv_out, pos, proj1_dup, proj2_dup, o_f16, total;
 };
 
 PreparedLayout prepared_layout(const aut_config *c) {
@@ -49,7 +49,7 @@ PreparedLayout prepared_layout(const aut_config *c) {
     p.pos = r.take((size_t)kTokensPerChunk * d * 4);
     p.proj1_dup = r.take(d * 2 * d * 2);
     p.proj2_dup = r.take((size_t)c->output_dim * 2 * d * 2);
-    p.o_dup = r.take((size_t)std::max(c->layers, 1) * d * 2 * d * 2);
+    p.o_f16 = r.take((size_t)std::max(c->layers, 1) * d * d * 2);
     p.total = r.off;
     return p;
 }
@@ -76,7 +76,7 @@ bool weights_complete(const aut_config *c, const aut_weights *w, int n_layers, b
     if (stem && (!w->conv1_w || !w->conv1_b || !w->conv2_b || !w->conv3_b || !w->conv2_w_tap ||
                  !w->conv3_w_tap || !w->conv_out_w_fc || !w->pos_table))
         return false;
-    if (n_layers > 0 && (!w->layers || !w->o_w_dup)) return false;
+    if (n_layers > 0 && (!w->layers || !w->o_w_f16)) return false;
     for (int i = 0; i < n_layers; ++i) {
         const aut_layer_weights &l = w->layers[i];
         if (!l.ln1_w || !l.ln1_b || !l.qkv_w || !l.qkv_b || !l.o_w || !l.o_b || !l.ln2_w ||
@@ -106,7 +106,8 @@ struct Ctx {
         if (i < trace->capacity) {
             if (trace->kinds) trace->kinds[i] = kind;
             if (trace->events &&
-                cudaEventRecord(static_cast<cudaEvent_t>(trace->events[i]), st) != cudaSuccess)
+                cudaEventRecordWithFlags(static_cast<cudaEvent_t>(trace->events[i]), st,
+                                         cudaEventRecordExternal) != cudaSuccess)
                 return AUT_ERR_CUDA;
         }
         return AUT_OK;
@@ -119,8 +120,9 @@ struct Ctx {
 };
 
 aut_status linear(const Ctx &c, const void *a, const void *w, const void *b, void *out, int M,
-                  int N, int K, int epi, int kind, int ldo = 0) {
+                  int N, int K, int epi, int kind, int ldo = 0, bool f16 = false) {
     LinearLaunch L{};
+    L.f16 = f16;
     L.a = a;
     L.w = w;
     L.bias = b;
@@ -243,9 +245,9 @@ aut_status run_encode(const Ctx &c, float *x, int T, int nW, int n_layers, void 
         AUT_TRY(cuda_status(launch_window_attention(qkv, attn, cu, nW, d, cfg->heads, c.st, T,
                                                     c.status)));
         AUT_TRY(c.mark(AUT_K_ATTENTION));
-        // attention output [hi | lo] against [o_w | o_w]
-        const void *o_w2 = static_cast<const uint8_t *>(c.w->o_w_dup) + (size_t)l * d * 2 * d * 2;
-        AUT_TRY(linear(c, attn, o_w2, lw.o_b, x, T, d, 2 * d, kEpiResidF32, AUT_K_O_PROJ));
+        // fp16 attention output against the fp16 copy of o_w
+        const void *o_w16 = static_cast<const uint8_t *>(c.w->o_w_f16) + (size_t)l * d * d * 2;
+        AUT_TRY(linear(c, attn, o_w16, lw.o_b, x, T, d, d, kEpiResidF32, AUT_K_O_PROJ, 0, true));
         AUT_TRY(cuda_status(launch_layernorm(x, lw.ln2_w, lw.ln2_b, xn, T, d, cfg->ln_eps, c.st)));
         AUT_TRY(c.mark(AUT_K_LAYERNORM));
         AUT_TRY(linear(c, xn, lw.fc1_w, lw.fc1_b, ffn, T, F, d, kEpiBf16Gelu, AUT_K_FC1));
@@ -306,7 +308,7 @@ WorkspaceLayout workspace_layout(const aut_config *c, int64_t T, int64_t nW, int
     Region a{base};
     L.xn = a.take((size_t)T * 2 * d * 2);  // [hi | lo] rows for the projector
     L.qkv = a.take((size_t)T * 3 * d * 2);
-    L.attn = a.take((size_t)T * 2 * d * 2);  // [hi | lo] rows
+    L.attn = a.take((size_t)T * d * 2);  // fp16
     L.ffn = a.take((size_t)T * std::max(F, 2 * d) * 2);
     const int G = (int)std::min<int64_t>(n_ch, c->conv_chunksize);
     L.group_chunks = G;
@@ -352,14 +354,13 @@ extern "C" aut_status aut_prepare_weights(const aut_config *cfg, const aut_weigh
     out.pos_table = base + p.pos;
     out.proj1_w_dup = base + p.proj1_dup;
     out.proj2_w_dup = base + p.proj2_dup;
-    out.o_w_dup = base + p.o_dup;
+    out.o_w_f16 = base + p.o_f16;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     for (int l = 0; l < cfg->layers; ++l) {
         if (!src->layers || !src->layers[l].o_w) return AUT_ERR_INVALID_ARG;
-        AUT_TRY(cuda_status(launch_duplicate_k(src->layers[l].o_w,
-                                               base + p.o_dup + (size_t)l * cfg->d_model * 2 *
-                                                                    cfg->d_model * 2,
-                                               cfg->d_model, cfg->d_model, st)));
+        AUT_TRY(cuda_status(launch_to_f16(src->layers[l].o_w,
+                                          base + p.o_f16 + (size_t)l * cfg->d_model * cfg->d_model * 2,
+                                          (size_t)cfg->d_model * cfg->d_model, st)));
     }
     AUT_TRY(cuda_status(launch_duplicate_k(src->proj1_w, base + p.proj1_dup, cfg->d_model,
                                            cfg->d_model, st)));
@@ -469,6 +470,7 @@ extern "C" aut_status aut_linear(const void *x, const void *w, const void *bias,
     L.timeout_ns = timeout_ms ? (unsigned long long)timeout_ms * 1000000ull : kDefaultTimeoutNs;
     L.fault_inject = (flags & AUT_LINEAR_FAULT_INJECT) ? 1 : 0;
     L.single_cta = (flags & AUT_LINEAR_SINGLE_CTA) != 0;
+    L.f16 = (flags & AUT_LINEAR_F16) != 0;
     return gemm_status(launch_linear(L, reinterpret_cast<cudaStream_t>(stream)));
 }
 

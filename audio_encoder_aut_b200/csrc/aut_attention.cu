@@ -4,23 +4,37 @@
 // (aut_encoder page, AuTAttention: block-diagonal over the packed windows, no
 // cache; openarchlab "1A . AuT Audio Encoder", section 3: non-causal within each
 // segment).  A window has at most 128 tokens, so one (window, head) is one
-// 128-row tile and the softmax is exact in one pass over the tile:
+// 128-row tile and the softmax is exact in one pass over the tile.
 //
-//   TMA:      Q, K, V tiles [128 x 64] bf16 (128-byte swizzle) from qkv [T, 3d];
-//             rows past the window's end are the next window's rows (or zero
-//             past T) and are masked below
-//   tcgen05:  S = Q K^T            M = 128, N = 128, K = 64 -> TMEM columns 0..127
-//   threads:  two warps per TMEM lane quadrant, each over half of the keys, own
-//             query row r: row max over the valid keys, then
-//             p = exp2((s - max) * log2(e) / sqrt(64)), row sum, and P written to
-//             shared memory as fp16 (P lies in [0, 1]; fp16 keeps 11 significant
-//             bits, 8x finer than bf16) in the swizzled K-major layout the MMA
-//             reads, over the Q and K tiles the first MMA no longer needs; V is
-//             converted in place to fp16 (exact for bf16 values in fp16's range)
-//   tcgen05:  O = P V              M = 128, N = 64, K = 128, f16 inputs, V read
-//                                  MN-major -> TMEM columns 0..63 (S is dead)
-//   threads:  O / rowsum written as [hi | lo] bf16 halves of a 2 d row (rows past
-//             the window's end are not written)
+// The kernel is persistent (two CTAs per SM) and walks the (window, head)
+// tiles with a grid stride.  Warp roles:
+//   warp 0     TMA producer: Q, K, V tiles [128 x 64] bf16 (128-byte swizzle)
+//              from qkv [T, 3d] into a ring of kStages stages; rows past the
+//              window's end are the next window's rows (or zero past T) and
+//              are masked below
+//   warp 1     MMA issuer:  S = Q K^T  (M = 128, N = window length rounded up
+//              to 16, K = 64) into TMEM columns 0..127; once P is ready,
+//              O = P V (M = 128, N = 64, K = window length rounded up to 16,
+//              fp16 inputs, V read MN-major) into TMEM columns 128..191
+//   warps 2-9  softmax and epilogue, two warps per TMEM lane quadrant, each
+//              over half of the keys: row max (exchanged between the two
+//              halves), p = exp2((s - max) * log2(e) / sqrt(64)) written to
+//              shared memory as fp16 (P lies in [0, 1]; fp16 keeps 11
+//              significant bits, 8x finer than bf16) in the swizzled K-major
+//              layout the MMA reads, over the Q and K tiles the first MMA no
+//              longer needs; V converted in place to fp16 (saturating: bf16
+//              values beyond fp16's range clamp to +-65504); then O / rowsum
+//              written as fp16 [T, d] (11 significant bits for the o_proj GEMM,
+//              which runs on fp16 operands; rows past the window's end are not
+//              written)
+// The producer runs up to kStages tiles ahead, so the loads of the next tiles
+// overlap the softmax and the stores of this one; the second CTA on the SM
+// fills the gaps of the first.
+//
+// Two TMEM users never share an SM between kernels of the forward: this
+// kernel's shared memory (about 100 KB) and the GEMM's (about 197 KB) exceed
+// the SM's 228 KB together, so a CTA launched early by programmatic dependent
+// launch cannot hold TMEM columns that a CTA of the previous kernel still needs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -35,21 +49,27 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 
-constexpr int kTile = 128;                 // query / key rows per tile
-constexpr int kHd = 64;                    // head dim (one 128-byte swizzle row)
+constexpr int kTile = 128;                   // query / key rows per tile
+constexpr int kHd = 64;                      // head dim (one 128-byte swizzle row)
 constexpr int kTileBytes = kTile * kHd * 2;  // 16 KiB
-// Shared memory: Q | K | V; P (fp16, 128 x 128) overwrites Q | K once S is done.
-constexpr int kOffQ = 0, kOffK = kTileBytes, kOffV = 2 * kTileBytes;
-constexpr int kOffRed = 3 * kTileBytes;               // row max / sum of the two column halves
+constexpr int kStages = 2;
+constexpr int kStageBytes = 3 * kTileBytes;  // Q | K | V; P (fp16, 128 x 128) overwrites Q | K
+constexpr int kOffRed = kStages * kStageBytes;  // row max and sum of the two key halves
 constexpr int kOffBar = kOffRed + 2 * 2 * kTile * 4;
-constexpr int kSmem = 1024 + kOffBar + 64;
-constexpr int kThreads = 256;  // 8 warps: TMEM lane quadrant x half of the key (or O) columns
-constexpr uint32_t kTmemCols = 128;        // S: 0..127, then O: 0..63
+// full[kStages], empty[kStages], s_full, p_full, o_full, o_empty, xchg[4], mma_done
+constexpr int kNumBars = 2 * kStages + 4 + 4 + 1;
+constexpr int kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
+constexpr int kComputeWarps = 8;
+constexpr int kThreads = 64 + 32 * kComputeWarps;
+constexpr int kCtasPerSm = 2;
+constexpr uint32_t kTmemCols = 256;  // S: 0..127, O: 128..191
+constexpr uint32_t kColO = 128;
+constexpr unsigned long long kTimeoutNs = 4000ull * 1000ull * 1000ull;
+
 // kind::f16 with fp16 A and B, fp32 accumulate, A K-major, B MN-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
     return (1u << 4) | (1u << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr unsigned long long kTimeoutNs = 4000ull * 1000ull * 1000ull;
 
 // Byte offset of the 16-byte chunk `chunk` (8 keys) of row `r` in a K-major
 // operand of 128 rows x 128 keys held as two 128-byte-swizzled atoms of 64 keys.
@@ -58,33 +78,55 @@ __device__ __forceinline__ uint32_t p_chunk_offset(int r, int chunk) {
     return (uint32_t)(atom * kTileBytes + r * 128 + ((c ^ (r & 7)) << 4));
 }
 
-__global__ void __launch_bounds__(kThreads) window_attn_tc_kernel(
-    const __grid_constant__ CUtensorMap tm_qkv, bf16 *__restrict__ out, const int *__restrict__ cu,
-    int d, float scale_log2e, int *status) {
+__device__ __forceinline__ void signal_abort(int *status, volatile int *abort) {
+    if (status) atomicCAS(status, 0, kDevTimeout);
+    *abort = 1;
+}
+
+// Tokens of window w (the last 16-row step of the MMAs covers the ragged end).
+__device__ __forceinline__ void window_of(const int *cu, int w, int *s0, int *len, int *n16) {
+    *s0 = cu[w];
+    *len = cu[w + 1] - *s0;
+    *n16 = max(1, (*len + 15) >> 4);
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_qkv, __half *__restrict__ out, const int *__restrict__ cu,
+    int n_windows, int heads, int d, float scale_log2e, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t *sQ = sm + kOffQ, *sK = sm + kOffK, *sV = sm + kOffV;
-    uint8_t *sP = sQ;  // reuses Q | K after the S MMAs completed
     float *red_max = reinterpret_cast<float *>(sm + kOffRed);  // [2 halves][128 rows]
     float *red_sum = red_max + 2 * kTile;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kOffBar);  // load, S done, O done
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 3);
-    volatile int *fail = reinterpret_cast<volatile int *>(tslot + 1);  // the load timed out
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int row = quad * 32 + lane;  // query row of this thread (TMEM lane)
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + kOffBar);
+    uint64_t *empty = full + kStages;
+    uint64_t *s_full = empty + kStages;  // S in TMEM
+    uint64_t *p_full = s_full + 1;       // P and fp16 V in shared memory, S read
+    uint64_t *o_full = p_full + 1;       // O in TMEM
+    uint64_t *o_empty = o_full + 1;      // O read out of TMEM
+    uint64_t *xchg = o_empty + 1;        // per lane quadrant: the two key halves met
+    uint64_t *mma_done = xchg + 4;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    int *abort_flag = reinterpret_cast<int *>(tslot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     pdl_trigger();
-    if (tid == 0) {
-        mbar_init(bar + 0, 1);
-        mbar_init(bar + 1, 1);
-        mbar_init(bar + 2, 1);
-        *fail = 0;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, kComputeWarps);
+        mbar_init(o_full, 1);
+        mbar_init(o_empty, kComputeWarps);
+        for (int q = 0; q < 4; ++q) mbar_init(xchg + q, 64);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tm_qkv);
     }
-    if (warp == 0) {
+    if (warp == 1) {
         tmem_alloc(tslot, kTmemCols);
         tmem_relinquish();
     }
@@ -92,146 +134,233 @@ __global__ void __launch_bounds__(kThreads) window_attn_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
+    volatile int *abort_v = abort_flag;
     pdl_wait();
+    const int n_tiles = n_windows * heads;
 
-    const int seg = blockIdx.x, h = blockIdx.y;
-    const int s0 = cu[seg], len = cu[seg + 1] - s0;
-    bool ok = len > 0;
-
-    if (ok && tid == 0) {
-        mbar_arrive_expect_tx(bar + 0, 3 * kTileBytes);
-        tma_load_2d(sQ, &tm_qkv, bar + 0, h * kHd, s0);
-        tma_load_2d(sK, &tm_qkv, bar + 0, d + h * kHd, s0);
-        tma_load_2d(sV, &tm_qkv, bar + 0, 2 * d + h * kHd, s0);
-        if (mbar_wait(bar + 0, 0, nullptr, kTimeoutNs)) {
-            tc_fence_after();
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kTile);
-#pragma unroll
-            for (int kk = 0; kk < kHd / 16; ++kk)
-                tc_mma_bf16(tmem, smem_desc_sw128(sQ) + 2 * kk, smem_desc_sw128(sK) + 2 * kk,
-                            idesc_s, kk > 0);
-            tc_commit(bar + 1);
-        } else {
-            if (status) atomicCAS(status, 0, kDevTimeout);
-            *fail = 1;  // nothing was issued to the tensor cores; release the row threads
-            mbar_arrive(bar + 1);
-        }
-    }
-
-    // ---- softmax of row `row` over the window's keys (two warps per row) ----
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    float row_sum = 1.f;
-    if (ok) {
-        if (!mbar_wait(bar + 1, 0, nullptr, kTimeoutNs)) {
-            if (status) atomicCAS(status, 0, kDevTimeout);
-        }
-        ok = *fail == 0;
-    }
-    tc_fence_after();
-    if (ok) {  // block-uniform: every thread shares `len`
-        float v[2][32];
-        tmem_ld32(trow + half * 64, v[0]);
-        tmem_ld32(trow + half * 64 + 32, v[1]);
-        tc_wait_ld();
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (half * 64 + c * 32 + j < len) mx = fmaxf(mx, v[c][j]);
-        red_max[half * kTile + row] = mx;
-        __syncthreads();
-        mx = fmaxf(red_max[row], red_max[kTile + row]);
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {  // 8 keys = one 16-byte chunk of P
-                uint32_t ph[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = q * 8 + 2 * e, key = half * 64 + c * 32 + j;
-                    const float p0 = key < len ? exp2f((v[c][j] - mx) * scale_log2e) : 0.f;
-                    const float p1 = key + 1 < len ? exp2f((v[c][j + 1] - mx) * scale_log2e) : 0.f;
-                    sum += p0 + p1;
-                    __half2 hp = __floats2half2_rn(p0, p1);
-                    ph[e] = *reinterpret_cast<uint32_t *>(&hp);
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer --
+            uint32_t issued = 0, parity = 0;
+            bool ok = true;
+            int k = 0;
+            for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++k) {
+                const int w = t / heads, h = t - w * heads;
+                const int s = k % kStages;
+                const uint32_t use = (uint32_t)(k / kStages);
+                if (k >= kStages && !mbar_wait(empty + s, (use - 1) & 1u, abort_v, kTimeoutNs)) {
+                    ok = false;
+                    break;
                 }
-                *reinterpret_cast<uint4 *>(sP + p_chunk_offset(row, half * 8 + c * 4 + q)) =
-                    make_uint4(ph[0], ph[1], ph[2], ph[3]);
+                uint8_t *st = sm + s * kStageBytes;
+                const int s0 = cu[w];
+                mbar_arrive_expect_tx(full + s, kStageBytes);
+                tma_load_2d(st, &tm_qkv, full + s, h * kHd, s0);
+                tma_load_2d(st + kTileBytes, &tm_qkv, full + s, d + h * kHd, s0);
+                tma_load_2d(st + 2 * kTileBytes, &tm_qkv, full + s, 2 * d + h * kHd, s0);
+                issued |= 1u << s;
+                parity = (parity & ~(1u << s)) | ((use & 1u) << s);
             }
+            if (!ok) signal_abort(status, abort_v);
+            // The last load issued on every stage has landed before the block may exit.
+            for (int s = 0; s < kStages; ++s)
+                if (issued >> s & 1u) mbar_wait(full + s, parity >> s & 1u, nullptr, kTimeoutNs);
         }
-        red_sum[half * kTile + row] = sum;
-        // V to fp16 in place (same positions, so the swizzled layout is kept).  Every
-        // thread acquires the TMA barrier (long complete) before reading V directly.
-        mbar_wait(bar + 0, 0, nullptr, kTimeoutNs);
-        uint4 *vv = reinterpret_cast<uint4 *>(sV) + tid * 4;
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // -------------------------------------------------- MMA issuer --
+            constexpr uint32_t idesc_o = idesc_f16_f32_bmn(kTile, kHd);
+            bool ok = true;
+            int k = 0;
+            for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++k) {
+                int s0, len, n16;
+                window_of(cu, t / heads, &s0, &len, &n16);
+                const int s = k % kStages;
+                const uint32_t use = (uint32_t)(k / kStages);
+                uint8_t *st = sm + s * kStageBytes;
+                if (!mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // S over the window's keys only (N = 16 n16 columns).
+                const uint32_t idesc_s = idesc_bf16_f32(kTile, 16 * n16);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            uint4 w = vv[u];
-            uint32_t *e = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&e[k]));
-                __half2 hv = __floats2half2_rn(f.x, f.y);
-                e[k] = *reinterpret_cast<uint32_t *>(&hv);
+                for (int kk = 0; kk < kHd / 16; ++kk)
+                    tc_mma_bf16(tmem, smem_desc_sw128(st) + 2 * kk,
+                                smem_desc_sw128(st + kTileBytes) + 2 * kk, idesc_s, kk > 0);
+                tc_commit(s_full);
+                if (!mbar_wait(p_full, k & 1u, abort_v, kTimeoutNs) ||
+                    (k > 0 && !mbar_wait(o_empty, (k - 1) & 1u, abort_v, kTimeoutNs))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // O = P V: k-step j covers keys 16 j .. 16 j + 16.
+                for (int j = 0; j < n16; ++j)
+                    tc_mma_bf16(tmem + kColO,
+                                smem_desc_sw128(st + (j >> 2) * kTileBytes) + 2 * (j & 3),
+                                smem_desc_sw128_mn(st + 2 * kTileBytes + j * 16 * 128), idesc_o,
+                                j > 0);
+                tc_commit(o_full);
+                tc_commit(empty + s);  // Q | K (now P) and V free once O is done
             }
-            vv[u] = w;
+            if (!ok) signal_abort(status, abort_v);
+            // Every MMA this thread issued has completed before TMEM is released.
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0, nullptr, kTimeoutNs);
         }
     } else {
-        __syncthreads();  // matches the row-max exchange above
-    }
-    fence_proxy_async_smem();  // P and V (generic-proxy writes) visible to the MMA
-    tc_fence_before();
-    __syncthreads();
-    if (ok) row_sum = red_sum[row] + red_sum[kTile + row];
-
-    if (ok && tid == 0) {
-        tc_fence_after();
-        // O = P V over 128 keys: k-step s covers keys 16 s .. 16 s + 16.
-        constexpr uint32_t idesc_o = idesc_f16_f32_bmn(kTile, kHd);
+        // --------------------------------------------- softmax, epilogue --
+        const int cw = warp - 2, ctid = threadIdx.x - 64;
+        const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
+        const int half = cw >> 2;   // keys [64 half, 64 half + 64); O columns [32 half, + 32)
+        const int row = quad * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        int k = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++k) {
+            const int w = t / heads, h = t - w * heads;
+            int s0, len, n16;
+            window_of(cu, w, &s0, &len, &n16);
+            const int s = k % kStages;
+            const uint32_t use = (uint32_t)(k / kStages);
+            uint8_t *st = sm + s * kStageBytes;
+            const bool active = quad * 32 < len;  // warp-uniform: some rows are valid
+            if (!mbar_wait(s_full, k & 1u, abort_v, kTimeoutNs)) {
+                signal_abort(status, abort_v);
+                break;
+            }
+            tc_fence_after();
+            // Row max over this warp's half of the keys.
+            float mx = -INFINITY;
+            if (active) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-            tc_mma_bf16(tmem, smem_desc_sw128(sP + (s >> 2) * kTileBytes) + 2 * (s & 3),
-                        smem_desc_sw128_mn(sV + s * 16 * 128), idesc_o, s > 0);
-        tc_commit(bar + 2);
-    }
-    if (ok) {
-        if (!mbar_wait(bar + 2, 0, nullptr, kTimeoutNs)) {
-            if (status) atomicCAS(status, 0, kDevTimeout);
-        }
-    }
-    tc_fence_after();
-    if (ok) {  // O columns half * 32 .. + 32 of row `row`
-        const float inv = 1.f / row_sum;
-        float v[32];
-        tmem_ld32(trow + half * 32, v);
-        tc_wait_ld();
-        if (row < len) {
-            bf16 *o = out + (size_t)(s0 + row) * 2 * d + h * kHd + half * 32;
+                for (int c = 0; c < 2; ++c) {
+                    const int key0 = half * 64 + c * 32;
+                    if (key0 < len) {  // uniform: the block shares `len`
+                        float v[32];
+                        tmem_ld32(trow + key0, v);
+                        tc_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a = v[q * 8 + 2 * e] * inv, b = v[q * 8 + 2 * e + 1] * inv;
-                    hi[e] = pack_bf16x2(a, b);
-                    const float2 hf =
-                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hi[e]));
-                    lo[e] = pack_bf16x2(a - hf.x, b - hf.y);
+                        for (int j = 0; j < 32; ++j)
+                            if (key0 + j < len) mx = fmaxf(mx, v[j]);
+                    }
                 }
-                *reinterpret_cast<uint4 *>(o + q * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(o + d + q * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            red_max[half * kTile + row] = mx;
+            mbar_arrive(xchg + quad);
+            if (!mbar_wait(xchg + quad, 0, abort_v, kTimeoutNs)) {
+                signal_abort(status, abort_v);
+                break;
+            }
+            mx = fmaxf(red_max[row], red_max[kTile + row]);
+            // P = exp of the scaled, shifted scores; zero past the window's end.
+            float sum = 0.f;
+            if (active) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int key0 = half * 64 + c * 32;
+                    if (key0 < len) {
+                        float v[32];
+                        tmem_ld32(trow + key0, v);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {  // 8 keys = one 16-byte chunk of P
+                            uint32_t ph[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = q * 8 + 2 * e;
+                                const float p0 =
+                                    key0 + j < len ? exp2f((v[j] - mx) * scale_log2e) : 0.f;
+                                const float p1 =
+                                    key0 + j + 1 < len ? exp2f((v[j + 1] - mx) * scale_log2e) : 0.f;
+                                sum += p0 + p1;
+                                __half2 hp = __floats2half2_rn(p0, p1);
+                                ph[e] = *reinterpret_cast<uint32_t *>(&hp);
+                            }
+                            *reinterpret_cast<uint4 *>(st + p_chunk_offset(row, key0 / 8 + q)) =
+                                make_uint4(ph[0], ph[1], ph[2], ph[3]);
+                        }
+                    }
+                }
+            }
+            red_sum[half * kTile + row] = sum;
+            // V rows the MMA reads, to fp16 in place (same positions, so the
+            // swizzled layout is kept).  Reading V directly needs the TMA
+            // barrier's phase observed by this thread (it completed long ago).
+            if (!mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs)) {
+                signal_abort(status, abort_v);
+                break;
+            }
+            {
+                uint4 *vv = reinterpret_cast<uint4 *>(st + 2 * kTileBytes);
+                for (int i = ctid; i < n16 * 128; i += 32 * kComputeWarps) {
+                    uint4 u = vv[i];
+                    uint32_t *e = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 f =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&e[m]));
+                        e[m] = pack_f16x2_sat(f.x, f.y);
+                    }
+                    vv[i] = u;
+                }
+            }
+            fence_proxy_async_smem();  // P and V (generic-proxy writes) visible to the MMA
+            tc_fence_before();         // S reads done before the next S overwrites it
+            mbar_arrive(xchg + quad);
+            if (!mbar_wait(xchg + quad, 1, abort_v, kTimeoutNs)) {
+                signal_abort(status, abort_v);
+                break;
+            }
+            const float inv = 1.f / (red_sum[row] + red_sum[kTile + row]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+            // Epilogue: O columns 32 half .. 32 half + 32 of row `row`.
+            if (!mbar_wait(o_full, k & 1u, abort_v, kTimeoutNs)) {
+                signal_abort(status, abort_v);
+                break;
+            }
+            tc_fence_after();
+            float o[32];
+            if (active) {
+                tmem_ld32(trow + kColO + half * 32, o);
+                tc_wait_ld();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_empty);
+            if (active && row < len) {
+                __half *dst = out + (size_t)(s0 + row) * d + h * kHd + half * 32;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pk[e] = pack_f16x2_sat(o[q * 8 + 2 * e] * inv, o[q * 8 + 2 * e + 1] * inv);
+                    *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
             }
         }
     }
-    if (tid == 0 && *fail) mbar_wait(bar + 0, 0, nullptr, kTimeoutNs);  // copies in flight land
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+int sm_count_cached() {
+    static int n[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!n[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 1;
+    }
+    return n[dev];
 }
 
 }  // namespace
@@ -255,8 +384,10 @@ cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu
     const uint32_t box[2] = {kHd, kTile};
     if (!make_tensor_map_bf16_sw128(&tm, 2, qkv, dims, strides, box)) return cudaErrorInvalidValue;
     const float scale_log2e = 1.4426950408889634f / 8.0f;  // log2(e) / sqrt(64)
-    return launch_pdl(window_attn_tc_kernel, dim3(n_windows, heads), dim3(kThreads), kSmem, st, 1, tm,
-                      static_cast<bf16 *>(out), cu_dev, d, scale_log2e, status);
+    const long tiles = (long)n_windows * heads;
+    const int grid = (int)std::min<long>(tiles, (long)kCtasPerSm * sm_count_cached());
+    return launch_pdl(window_attn_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, 1, tm,
+                      static_cast<__half *>(out), cu_dev, n_windows, heads, d, scale_log2e, status);
 }
 
 }  // namespace aut

@@ -162,9 +162,12 @@ GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
     const cuuint32_t ba[2] = {64, 128};
     const cuuint64_t db[2] = {(cuuint64_t)L.K, (cuuint64_t)L.N};
     const cuuint32_t bb[2] = {64, (cuuint32_t)(bn / cg)};
+    // fp16 operands use the same maps: the copies move bytes, and the zero fill
+    // of out-of-range rows is zero in both types.
     if (!make_map(&ta, 2, L.a, da, sa, ba) || !make_map(&tb, 2, L.w, db, sa, bb))
         return GemmStatus::kTensorMap;
     GemmArgs args{};
+    args.f16 = L.f16 ? 1 : 0;
     args.M = L.M;
     args.N = L.N;
     args.num_m_tiles = (L.M + 128 * cg - 1) / (128 * cg);

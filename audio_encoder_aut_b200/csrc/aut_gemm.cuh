@@ -35,6 +35,7 @@ constexpr int kGemmThreads = 64 + 32 * kEpilogueWarps;  // producer warp, MMA wa
 
 struct GemmArgs {
     int M, N;
+    int f16;  // A and B are fp16 (1) or bf16 (0)
     int num_m_tiles, num_n_tiles, num_k_blocks;
     // implicit-GEMM convolution operand (conv = 1)
     int conv;
@@ -269,7 +270,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // -------------------------------------------------- MMA issuer --
-            constexpr uint32_t idesc = idesc_bf16_f32(128 * CG, BN);
+            const uint32_t idesc =
+                args.f16 ? idesc_f16_f32(128 * CG, BN) : idesc_bf16_f32(128 * CG, BN);
             constexpr uint16_t kPair = 0x3;
             const bool resid_mode = args.epi == kEpiResidF32;
             int stage = 0, it = 0;

@@ -1,6 +1,7 @@
 // Non-GEMM kernels of the encoder: conv1 of the stem, LayerNorm, window
 // attention, one-time weight preparation, and small helpers.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "aut_internal.h"
@@ -241,13 +242,13 @@ AUT_DEV void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint3
 // whole and the softmax is exact in one pass: S = Q K^T (fp32), row max, exp,
 // row sum, O = P V / sum.  Keys past the window's length are masked; rows past it
 // are computed on zeros and not written.  Each of the 8 warps owns 16-row query
-// tiles.  P and the output carry a second bf16 term (hi + lo): the o_proj GEMM
-// that consumes the output then sees it to about 16 significant bits.
+// tiles.  P carries a second bf16 term (hi + lo); the output is fp16, which the
+// o_proj GEMM consumes with fp16 weights (11 significant bits).
 constexpr int kAttnWarps = 8;
 
 template <int HD>
 __global__ void __launch_bounds__(32 * kAttnWarps) window_attn_kernel(const bf16 *__restrict__ qkv,
-                                                          bf16 *__restrict__ out,
+                                                          __half *__restrict__ out,
                                                           const int *__restrict__ cu, int d,
                                                           float scale_log2e) {
     constexpr int LD = HD + 8;  // padded row: conflict-free ldmatrix
@@ -380,28 +381,18 @@ __global__ void __launch_bounds__(32 * kAttnWarps) window_attn_kernel(const bf16
                 }
             }
         }
-        // O / rowsum written as [hi | lo] bf16 halves of a 2 d row.
+        // O / rowsum written as fp16 [T, d] (saturating at +-65504).
         const float inv0 = 1.f / sum0, inv1 = 1.f / sum1;
         const int r0 = mt * 16 + g, r1 = r0 + 8;
 #pragma unroll
         for (int j = 0; j < HD / 8; ++j) {
             const int col = h * HD + j * 8 + 2 * t;
-            if (r0 < len) {
-                const float a = o_acc[j][0] * inv0, b = o_acc[j][1] * inv0;
-                const uint32_t hi = pack_bf16x2(a, b);
-                const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hi));
-                bf16 *o = out + (size_t)(s0 + r0) * 2 * d + col;
-                *reinterpret_cast<uint32_t *>(o) = hi;
-                *reinterpret_cast<uint32_t *>(o + d) = pack_bf16x2(a - hf.x, b - hf.y);
-            }
-            if (r1 < len) {
-                const float a = o_acc[j][2] * inv1, b = o_acc[j][3] * inv1;
-                const uint32_t hi = pack_bf16x2(a, b);
-                const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&hi));
-                bf16 *o = out + (size_t)(s0 + r1) * 2 * d + col;
-                *reinterpret_cast<uint32_t *>(o) = hi;
-                *reinterpret_cast<uint32_t *>(o + d) = pack_bf16x2(a - hf.x, b - hf.y);
-            }
+            if (r0 < len)
+                *reinterpret_cast<uint32_t *>(out + (size_t)(s0 + r0) * d + col) =
+                    pack_f16x2_sat(o_acc[j][0] * inv0, o_acc[j][1] * inv0);
+            if (r1 < len)
+                *reinterpret_cast<uint32_t *>(out + (size_t)(s0 + r1) * d + col) =
+                    pack_f16x2_sat(o_acc[j][2] * inv1, o_acc[j][3] * inv1);
         }
     }
 }
@@ -514,7 +505,7 @@ cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void 
 }
 
 template <int HD>
-cudaError_t run_window_attention(const bf16 *q, bf16 *o, const int *cu_dev, int n_windows, int d,
+cudaError_t run_window_attention(const bf16 *q, __half *o, const int *cu_dev, int n_windows, int d,
                                  int heads, float scale_log2e, cudaStream_t st) {
     constexpr int smem = 2 * kMaxWindowTokens * (HD + 8) * (int)sizeof(bf16);
     static bool attr_done[64] = {};
@@ -538,7 +529,7 @@ cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_de
         return launch_window_attention_tc(qkv, out, cu_dev, n_windows, d, heads, T, status, st);
     const float scale_log2e = 1.4426950408889634f / sqrtf((float)hd);
     const bf16 *q = static_cast<const bf16 *>(qkv);
-    bf16 *o = static_cast<bf16 *>(out);
+    __half *o = static_cast<__half *>(out);
     switch (hd) {
         case 16: return run_window_attention<16>(q, o, cu_dev, n_windows, d, heads, scale_log2e, st);
         case 32: return run_window_attention<32>(q, o, cu_dev, n_windows, d, heads, scale_log2e, st);
@@ -564,6 +555,22 @@ __global__ void duplicate_k_kernel(const bf16 *__restrict__ src, bf16 *__restric
 cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st) {
     duplicate_k_kernel<<<592, 256, 0, st>>>(static_cast<const bf16 *>(src), static_cast<bf16 *>(dst),
                                             N, K);
+    return cudaGetLastError();
+}
+
+// bf16 -> fp16 (saturating), n elements, n a multiple of 2.
+__global__ void to_f16_kernel(const bf16 *__restrict__ src, uint32_t *__restrict__ dst, size_t n2) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n2;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162 *>(src)[i]);
+        dst[i] = pack_f16x2_sat(f.x, f.y);
+    }
+}
+
+cudaError_t launch_to_f16(const void *src, void *dst, size_t n, cudaStream_t st) {
+    if (n % 2) return cudaErrorInvalidValue;
+    to_f16_kernel<<<592, 256, 0, st>>>(static_cast<const bf16 *>(src), static_cast<uint32_t *>(dst),
+                                       n / 2);
     return cudaGetLastError();
 }
 

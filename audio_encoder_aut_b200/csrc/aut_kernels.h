@@ -64,6 +64,7 @@ cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, i
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
                              float eps, cudaStream_t st, bool split = false);
 cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st);
+cudaError_t launch_to_f16(const void *src, void *dst, size_t n, cudaStream_t st);
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                     int d, int heads, cudaStream_t st, int T = -1,
                                     int *status = nullptr);
@@ -83,8 +84,8 @@ cudaError_t launch_upload(const int32_t *host_words, size_t n, int32_t *dst, cud
 enum class GemmStatus { kOk, kBadShape, kTensorMap, kLaunch };
 
 struct LinearLaunch {
-    const void *a;     // bf16 [M, K]
-    const void *w;     // bf16 [N, K]
+    const void *a;     // bf16 (fp16 with f16) [M, K]
+    const void *w;     // bf16 (fp16 with f16) [N, K]
     const void *bias;  // bf16 [N] or null
     void *out;
     int M, N, K, ldo;
@@ -97,6 +98,7 @@ struct LinearLaunch {
     unsigned long long timeout_ns;
     int fault_inject;
     bool single_cta = false;  // force one CTA per MMA (no CTA pairs)
+    bool f16 = false;         // A and W are fp16 instead of bf16
 };
 GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st);
 

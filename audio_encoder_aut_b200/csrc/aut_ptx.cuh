@@ -223,6 +223,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            ((uint32_t)(M >> 4) << 24);
 }
 
+// The same for fp16 A and B (a_format = b_format = 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Two floats to fp16x2 (round to nearest; beyond fp16's range clamps to
+// +-65504 instead of becoming infinite); `a` lands at the lower address.
+AUT_DEV uint32_t pack_f16x2_sat(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+
 // Programmatic dependent launch: let the next kernel in the stream start its
 // launch and set-up now; and wait until the previous kernel has completed and
 // its memory is visible.  Every kernel of the forward waits before its first

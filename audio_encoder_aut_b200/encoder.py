@@ -127,14 +127,16 @@ class Encoder:
         return out
 
     def capture(self, features: torch.Tensor, feature_lens, out: torch.Tensor | None = None,
-                warmup: int = 2):
+                warmup: int = 2, trace: A.aut_trace | None = None):
         """Records one aut_encode of this exact batch shape into a CUDA graph and
         returns (graph, out).  The plan is built on the host once, outside the
         graph (aut_encoder page, module docstring: the runner's plan is built
         outside the graph so the block loop replays as a CUDA graph); replaying
         the graph re-runs the whole forward on whatever `features` then holds.
         The graph keeps this encoder's workspace, so it must not be replayed
-        concurrently with another call on the same encoder."""
+        concurrently with another call on the same encoder.  With `trace`, the
+        graph also records trace.events[i] after launch i (an event node between
+        launches, which orders them fully: no launch overlaps its predecessor)."""
         if out is None:
             _, _, total, _, _ = self.plan(feature_lens)
             out = torch.empty((total, self.cfg.output_dim), dtype=torch.float32, device=self.device)
@@ -147,7 +149,7 @@ class Encoder:
         torch.cuda.synchronize(self.device)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side):
-            self.encode(features, feature_lens, out=out)
+            self.encode(features, feature_lens, out=out, trace=trace)
         return graph, out
 
     def check(self) -> int:

@@ -38,6 +38,13 @@ METRIC = "encoded audio-seconds/s on 1 B200 (bf16); tokens/s and % of bf16 TC pe
 UNIT = "audio-s/s"
 
 
+# DRAM bytes (read + write) per gemm_tc_kernel launch, mean over the 101 GEMM
+# launches of one omni_16req forward, from one ncu capture of this kernel
+# version (dram__bytes_read.sum + dram__bytes_write.sum, cold caches).  None
+# whenever the kernel has changed since that capture.
+GEMM_DRAM_BYTES_PER_LAUNCH = 45.36e6
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -241,30 +248,37 @@ def our_arm(args, rank, world, local_rank):
     flops, gemm_flops = credited_flops(cfg, lens, cu)
     pk, pk_sus, hbm, pk_src = peaks()
 
-    # Per-kernel breakdown from traced steps (events recorded between launches).
+    # Per-kernel breakdown: the same forward captured as a graph with an event
+    # node after every launch, replayed like the timed steps (L2 flushed first).
+    # The first launch's time counts from an event recorded just before the replay.
     cap = 4096
-    events = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(cap + 1)]
     for e in events:  # torch creates the CUDA event on first record
         e.record(stream)
     torch.cuda.synchronize()
-    ev_ptrs = (A.c_void_p * cap)(*[e.cuda_event for e in events])
+    ev_ptrs = (A.c_void_p * cap)(*[e.cuda_event for e in events[1:]])
     kinds = (A.c_int32 * cap)()
     trace = A.aut_trace(ev_ptrs, cap, 0, kinds)
+    if args.graph:
+        tgraph, _ = enc.capture(fd, lens, out=out, trace=trace)
+        traced_step = tgraph.replay
+    else:
+        def traced_step():
+            enc.encode(fd, lens, out=out, trace=trace)
+        traced_step()
+        torch.cuda.synchronize()
+    launches = trace.count
+    assert 0 < launches <= cap
     per_kind = {}
-    launches = 0
-    n_trace = max(1, min(3, args.steps))
+    n_trace = max(3, min(10, args.steps))
     for _ in range(n_trace):
         flush.zero_()
-        start = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-        enc.encode(fd, lens, out=out, trace=trace)
+        events[0].record(stream)
+        traced_step()
         torch.cuda.synchronize()
-        launches = trace.count
-        prev = start
-        for i in range(min(trace.count, cap)):
+        for i in range(launches):
             k = A.KERNEL_KINDS[kinds[i]]
-            per_kind.setdefault(k, []).append(prev.elapsed_time(events[i]))
-            prev = events[i]
+            per_kind.setdefault(k, []).append(events[i].elapsed_time(events[i + 1]))
     kind_ms = {k: sum(v) / n_trace for k, v in per_kind.items()}
     gemm_launches = sum(len(v) for k, v in per_kind.items() if k in A.GEMM_KINDS) / n_trace
     gemm_ms = sum(kind_ms[k] for k in kind_ms if k in A.GEMM_KINDS)
@@ -325,7 +339,9 @@ def our_arm(args, rank, world, local_rank):
                          "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
                          "frac": achieved / pk, "peak_source": f"{pk_src} bf16 burst",
                          "peak_sustained": pk_sus, "launches_per_step": gemm_launches,
-                         "avg_launch_ms": gemm_avg_ms, "traffic": None},
+                         "avg_launch_ms": gemm_avg_ms, "traffic": GEMM_DRAM_BYTES_PER_LAUNCH,
+                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + "
+                                         "dram__bytes_write.sum, mean over one forward's GEMMs)"},
             "kernel_ms_per_step": {k: round(v, 4) for k, v in sorted(kind_ms.items(), key=lambda x: -x[1])},
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": h_feats.numel() * h_feats.element_size(),

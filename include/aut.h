@@ -92,7 +92,8 @@ typedef struct {
      * two-term (hi + lo bf16) projector operands. */
     const void *conv2_w_tap, *conv3_w_tap, *conv_out_w_fc, *pos_table;
     const void *proj1_w_dup, *proj2_w_dup;
-    const void *o_w_dup; /* [layers][d][2d]: every layer's o_proj weight repeated along K */
+    const void *o_w_f16; /* fp16 [layers][d][d]: every layer's o_proj weight in fp16 (the
+                          * operand type of the attention output) */
 } aut_weights;
 
 /* aut_encoder page, AuTEncoder.layout / AuTEncoderConfig.tokens_for_frames /
@@ -160,7 +161,9 @@ typedef enum {
  * cudaEvent_t handles (NULL with capacity 0 to only count); kinds: int32
  * [capacity] or NULL.  The library records events[i] on the stream right after
  * its i-th kernel launch and stores the kernel's aut_kernel_kind in kinds[i];
- * count receives the number of kernels launched (even beyond capacity). */
+ * count receives the number of kernels launched (even beyond capacity).  The
+ * records are external (cudaEventRecordExternal), so under stream capture they
+ * become event-record nodes of the graph, re-recorded on every replay. */
 typedef struct {
     void **events;
     int32_t capacity;
@@ -205,9 +208,11 @@ aut_status aut_encode_packed(const aut_config *cfg, const aut_weights *prepared,
  * (0 = default of 4000 ms).  flags: AUT_LINEAR_FAULT_INJECT makes the first block
  * skip its first operand load so that its consumer's wait runs out (tests of the
  * timeout path only); AUT_LINEAR_SINGLE_CTA keeps every MMA on one SM (no CTA
- * pairs); 0 for normal use. */
+ * pairs); AUT_LINEAR_F16 takes x and w as fp16 instead of bf16 (the o_proj
+ * GEMM over the fp16 attention output); 0 for normal use. */
 #define AUT_LINEAR_FAULT_INJECT 1
 #define AUT_LINEAR_SINGLE_CTA 2
+#define AUT_LINEAR_F16 4
 aut_status aut_linear(const void *x, const void *w, const void *bias, void *y, int32_t M,
                       int32_t N, int32_t K, int32_t epilogue, int32_t *status,
                       int32_t timeout_ms, int32_t flags, aut_stream_t stream);
@@ -222,9 +227,10 @@ aut_status aut_layernorm(const void *x, const void *gamma, const void *beta, voi
 /* Window attention (aut_encoder page, AuTAttention; openarchlab "1A . AuT Audio
  * Encoder", section 3: non-causal attention limited to each cu_seqlens segment):
  * for every segment and head, softmax(Q K^T / sqrt(hd)) V.  qkv: device bf16
- * [T, 3 d] (q | k | v); out: device bf16 [T, 2 d], each row [hi | lo] with
- * hi = bf16(o) and lo = bf16(o - hi), so hi + lo carries o to about 16
- * significant bits (P is likewise applied as two bf16 terms).  cu_seqlens: HOST int32
+ * [T, 3 d] (q | k | v); out: device fp16 [T, d] (11 significant bits, 8x
+ * finer than bf16; values beyond +-65504 saturate), the operand of the fp16
+ * o_proj GEMM.  The probabilities P enter the P V product as fp16 for head_dim
+ * 64 (tensor-core path) and as two bf16 terms otherwise.  cu_seqlens: HOST int32
  * [num_windows + 1], every window at most 128 tokens.  workspace: device, at
  * least 4 * (num_windows + 1) bytes (the uploaded cu_seqlens). */
 aut_status aut_window_attention(const void *qkv, void *out, int32_t T, int32_t d, int32_t heads,

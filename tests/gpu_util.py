@@ -28,15 +28,21 @@ def assert_rows_close(got, ref, what="", cos_min=COS_MIN, rel_max=REL_MAX):
     return cos.min(), rel.max()
 
 
-def assert_bf16_output_close(got, ref, what="", atol=None):
+def assert_bf16_output_close(got, ref, what="", atol=None, rel=2.0 ** -8, kind="bf16"):
     """Bound for a kernel whose output is stored in bf16 from fp32 arithmetic:
-    round-to-nearest-even to 8 significant bits errs by at most 2^-8 |v|, plus a
-    small absolute term for the fp32 arithmetic (default 1e-3 of the row RMS)."""
+    round-to-nearest-even to 8 significant bits errs by at most 2^-8 |v| (rel),
+    plus a small absolute term for the fp32 arithmetic (default 1e-3 of the row
+    RMS)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if atol is None:
         atol = 1e-3 * np.sqrt((ref ** 2).mean(1, keepdims=True))
-    excess = np.abs(got - ref) - (2.0 ** -8 * np.abs(ref) + atol)
+    excess = np.abs(got - ref) - (rel * np.abs(ref) + atol)
     i = np.unravel_index(int(np.argmax(excess)), excess.shape)
     assert excess.max() <= 0, (f"{what}: element {i} got {got[i]:.6g} ref {ref[i]:.6g} "
-                               f"exceeds the bf16 bound by {excess[i]:.3g}")
+                               f"exceeds the {kind} bound by {excess[i]:.3g}")
+
+
+def assert_f16_output_close(got, ref, what="", atol=None):
+    """The same for an fp16 output: 11 significant bits, at most 2^-11 |v|."""
+    assert_bf16_output_close(got, ref, what, atol, rel=2.0 ** -11, kind="fp16")

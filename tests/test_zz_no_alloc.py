@@ -31,8 +31,8 @@ def test_noalloc_attention_matches_workspace_attention_on_two_calls():
         rng = np.random.default_rng(100 + call)
         qkv = torch.from_numpy(S.round_bf16(rng.standard_normal((T, 3 * d)).astype(np.float32)))
         qkv = qkv.to("cuda").to(torch.bfloat16)
-        ref = torch.zeros((T, 2 * d), dtype=torch.bfloat16, device="cuda")
-        got = torch.full((T, 2 * d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ref = torch.zeros((T, d), dtype=torch.float16, device="cuda")
+        got = torch.full((T, d), float("nan"), dtype=torch.float16, device="cuda")
         ws = torch.empty(4 * (len(cu) + 1), dtype=torch.uint8, device="cuda")
         assert A.aut_window_attention(qkv.data_ptr(), ref.data_ptr(), T, d, heads, cu,
                                       ws.data_ptr(), ws.numel(), st) == A.AUT_OK
