@@ -15,7 +15,9 @@
 //   warp 1     MMA issuer:  S = Q K^T  (M = 128, N = window length rounded up
 //              to 16, K = 64) into TMEM columns 0..127; once P is ready,
 //              O = P V (M = 128, N = 64, K = window length rounded up to 16,
-//              fp16 inputs, V read MN-major) into TMEM columns 128..191
+//              fp16 inputs, V read MN-major) into one of two O buffers (TMEM
+//              columns 128..191 and 192..255), so tile k's softmax overlaps
+//              the O product of tile k - 1
 //   warps 2-9  softmax and epilogue, two warps per TMEM lane quadrant, each
 //              over half of the keys: row max (exchanged between the two
 //              halves), p = exp2((s - max) * log2(e) / sqrt(64)) written to
@@ -56,13 +58,13 @@ constexpr int kStages = 2;
 constexpr int kStageBytes = 3 * kTileBytes;  // Q | K | V; P (fp16, 128 x 128) overwrites Q | K
 constexpr int kOffRed = kStages * kStageBytes;  // row max and sum of the two key halves
 constexpr int kOffBar = kOffRed + 2 * 2 * kTile * 4;
-// full[kStages], empty[kStages], s_full, p_full, o_full, o_empty, xchg[4], mma_done
-constexpr int kNumBars = 2 * kStages + 4 + 4 + 1;
+// full[kStages], empty[kStages], s_full, p_full, o_full[2], o_empty[2], mma_done
+constexpr int kNumBars = 2 * kStages + 2 + 4 + 1;
 constexpr int kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
 constexpr int kComputeWarps = 8;
 constexpr int kThreads = 64 + 32 * kComputeWarps;
 constexpr int kCtasPerSm = 2;
-constexpr uint32_t kTmemCols = 256;  // S: 0..127, O: 128..191
+constexpr uint32_t kTmemCols = 256;  // S: 0..127, O: two buffers at 128..191 and 192..255
 constexpr uint32_t kColO = 128;
 constexpr unsigned long long kTimeoutNs = 4000ull * 1000ull * 1000ull;
 
@@ -76,6 +78,31 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
 __device__ __forceinline__ uint32_t p_chunk_offset(int r, int chunk) {
     const int atom = chunk >> 3, c = chunk & 7;
     return (uint32_t)(atom * kTileBytes + r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Named barrier ID over the 64 threads of two warps that also ORs their `fail`
+// flags: both warps get the same answer, so they leave a loop together.
+template <int ID>
+__device__ __forceinline__ bool sync_any_64(bool fail) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, 64, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)fail), "n"(ID)
+        : "memory");
+    return r != 0;
+}
+// The barrier of lane quadrant `quad` (ids 1-4; 0 is __syncthreads).
+__device__ __forceinline__ bool quad_sync_any(int quad, bool fail) {
+    switch (quad) {
+        case 0: return sync_any_64<1>(fail);
+        case 1: return sync_any_64<2>(fail);
+        case 2: return sync_any_64<3>(fail);
+        default: return sync_any_64<4>(fail);
+    }
 }
 
 __device__ __forceinline__ void signal_abort(int *status, volatile int *abort) {
@@ -102,10 +129,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
     uint64_t *empty = full + kStages;
     uint64_t *s_full = empty + kStages;  // S in TMEM
     uint64_t *p_full = s_full + 1;       // P and fp16 V in shared memory, S read
-    uint64_t *o_full = p_full + 1;       // O in TMEM
-    uint64_t *o_empty = o_full + 1;      // O read out of TMEM
-    uint64_t *xchg = o_empty + 1;        // per lane quadrant: the two key halves met
-    uint64_t *mma_done = xchg + 4;
+    uint64_t *o_full = p_full + 1;       // [2] O buffer in TMEM
+    uint64_t *o_empty = o_full + 2;      // [2] O buffer read out of TMEM
+    uint64_t *mma_done = o_empty + 2;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(mma_done + 1);
     int *abort_flag = reinterpret_cast<int *>(tslot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,9 +144,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
         }
         mbar_init(s_full, 1);
         mbar_init(p_full, kComputeWarps);
-        mbar_init(o_full, 1);
-        mbar_init(o_empty, kComputeWarps);
-        for (int q = 0; q < 4; ++q) mbar_init(xchg + q, 64);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(o_full + b, 1);
+            mbar_init(o_empty + b, kComputeWarps);
+        }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -190,19 +217,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
                     tc_mma_bf16(tmem, smem_desc_sw128(st) + 2 * kk,
                                 smem_desc_sw128(st + kTileBytes) + 2 * kk, idesc_s, kk > 0);
                 tc_commit(s_full);
+                // O buffer k & 1 was last drained by the epilogue of tile k - 2.
+                const int ob = k & 1;
                 if (!mbar_wait(p_full, k & 1u, abort_v, kTimeoutNs) ||
-                    (k > 0 && !mbar_wait(o_empty, (k - 1) & 1u, abort_v, kTimeoutNs))) {
+                    (k >= 2 && !mbar_wait(o_empty + ob, ((k - 2) >> 1) & 1u, abort_v, kTimeoutNs))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 // O = P V: k-step j covers keys 16 j .. 16 j + 16.
                 for (int j = 0; j < n16; ++j)
-                    tc_mma_bf16(tmem + kColO,
+                    tc_mma_bf16(tmem + kColO + ob * kHd,
                                 smem_desc_sw128(st + (j >> 2) * kTileBytes) + 2 * (j & 3),
                                 smem_desc_sw128_mn(st + 2 * kTileBytes + j * 16 * 128), idesc_o,
                                 j > 0);
-                tc_commit(o_full);
+                tc_commit(o_full + ob);
                 tc_commit(empty + s);  // Q | K (now P) and V free once O is done
             }
             if (!ok) signal_abort(status, abort_v);
@@ -212,45 +241,81 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
         }
     } else {
         // --------------------------------------------- softmax, epilogue --
+        // Tile k's softmax runs while the tensor cores finish O of tile k - 1
+        // (two O buffers); tile k - 1's epilogue follows, by which time S of
+        // tile k + 1 is being computed.  The two warps of a lane quadrant meet at
+        // a named barrier that also ORs their failure flags, so both leave the
+        // loop together after a time-out.
         const int cw = warp - 2, ctid = threadIdx.x - 64;
         const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
         const int half = cw >> 2;   // keys [64 half, 64 half + 64); O columns [32 half, + 32)
         const int row = quad * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        int k = 0;
-        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++k) {
+        bool fail = false;
+        // Epilogue of local tile kk (global tile t): O / rowsum to fp16 rows.
+        auto epilogue = [&](int kk, int t, float inv) {
             const int w = t / heads, h = t - w * heads;
             int s0, len, n16;
             window_of(cu, w, &s0, &len, &n16);
+            const int ob = kk & 1;
+            fail = fail || !mbar_wait(o_full + ob, (kk >> 1) & 1u, abort_v, kTimeoutNs);
+            fail = __any_sync(0xffffffffu, fail);
+            if (fail) return;
+            tc_fence_after();
+            const bool active = quad * 32 < len;
+            float o[32];
+            if (active) {
+                tmem_ld32(trow + kColO + ob * kHd + half * 32, o);
+                tc_wait_ld();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_empty + ob);
+            if (active && row < len) {
+                __half *dst = out + (size_t)(s0 + row) * d + h * kHd + half * 32;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pk[e] = pack_f16x2_sat(o[q * 8 + 2 * e] * inv, o[q * 8 + 2 * e + 1] * inv);
+                    *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        };
+        int k = 0, prev_t = -1;
+        float prev_inv = 0.f;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++k) {
+            int s0, len, n16;
+            window_of(cu, t / heads, &s0, &len, &n16);
             const int s = k % kStages;
             const uint32_t use = (uint32_t)(k / kStages);
             uint8_t *st = sm + s * kStageBytes;
             const bool active = quad * 32 < len;  // warp-uniform: some rows are valid
-            if (!mbar_wait(s_full, k & 1u, abort_v, kTimeoutNs)) {
-                signal_abort(status, abort_v);
-                break;
-            }
-            tc_fence_after();
-            // Row max over this warp's half of the keys.
+            fail = fail || !mbar_wait(s_full, k & 1u, abort_v, kTimeoutNs);
+            fail = __any_sync(0xffffffffu, fail);
             float mx = -INFINITY;
-            if (active) {
+            if (!fail) {
+                tc_fence_after();
+                // Row max over this warp's half of the keys.
+                if (active) {
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int key0 = half * 64 + c * 32;
-                    if (key0 < len) {  // uniform: the block shares `len`
-                        float v[32];
-                        tmem_ld32(trow + key0, v);
-                        tc_wait_ld();
+                    for (int c = 0; c < 2; ++c) {
+                        const int key0 = half * 64 + c * 32;
+                        if (key0 < len) {  // uniform: the block shares `len`
+                            float v[32];
+                            tmem_ld32(trow + key0, v);
+                            tc_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (key0 + j < len) mx = fmaxf(mx, v[j]);
+                            for (int j = 0; j < 32; ++j)
+                                if (key0 + j < len) mx = fmaxf(mx, v[j]);
+                        }
                     }
                 }
+                red_max[half * kTile + row] = mx;
             }
-            red_max[half * kTile + row] = mx;
-            mbar_arrive(xchg + quad);
-            if (!mbar_wait(xchg + quad, 0, abort_v, kTimeoutNs)) {
-                signal_abort(status, abort_v);
+            if (quad_sync_any(quad, fail)) {
+                fail = true;
                 break;
             }
             mx = fmaxf(red_max[row], red_max[kTile + row]);
@@ -288,11 +353,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
             // V rows the MMA reads, to fp16 in place (same positions, so the
             // swizzled layout is kept).  Reading V directly needs the TMA
             // barrier's phase observed by this thread (it completed long ago).
-            if (!mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs)) {
-                signal_abort(status, abort_v);
-                break;
-            }
-            {
+            fail = !mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs);
+            if (!fail) {
                 uint4 *vv = reinterpret_cast<uint4 *>(st + 2 * kTileBytes);
                 for (int i = ctid; i < n16 * 128; i += 32 * kComputeWarps) {
                     uint4 u = vv[i];
@@ -308,40 +370,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
             }
             fence_proxy_async_smem();  // P and V (generic-proxy writes) visible to the MMA
             tc_fence_before();         // S reads done before the next S overwrites it
-            mbar_arrive(xchg + quad);
-            if (!mbar_wait(xchg + quad, 1, abort_v, kTimeoutNs)) {
-                signal_abort(status, abort_v);
+            if (quad_sync_any(quad, fail)) {
+                fail = true;
                 break;
             }
             const float inv = 1.f / (red_sum[row] + red_sum[kTile + row]);
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
-            // Epilogue: O columns 32 half .. 32 half + 32 of row `row`.
-            if (!mbar_wait(o_full, k & 1u, abort_v, kTimeoutNs)) {
-                signal_abort(status, abort_v);
-                break;
-            }
-            tc_fence_after();
-            float o[32];
-            if (active) {
-                tmem_ld32(trow + kColO + half * 32, o);
-                tc_wait_ld();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(o_empty);
-            if (active && row < len) {
-                __half *dst = out + (size_t)(s0 + row) * d + h * kHd + half * 32;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        pk[e] = pack_f16x2_sat(o[q * 8 + 2 * e] * inv, o[q * 8 + 2 * e + 1] * inv);
-                    *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
+            // Tile k - 1's output, while O of tile k and S of tile k + 1 compute.
+            if (prev_t >= 0) epilogue(k - 1, prev_t, prev_inv);
+            prev_t = t;
+            prev_inv = inv;
         }
+        if (!fail && prev_t >= 0) epilogue(k - 1, prev_t, prev_inv);
+        if (fail) signal_abort(status, abort_v);
     }
     tc_fence_before();
     __syncthreads();

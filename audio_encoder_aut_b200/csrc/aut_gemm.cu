@@ -35,11 +35,12 @@ EncodeTiledFn encode_fn() {
 // bf16 tensor map with 128-byte swizzle; dims innermost first, strides in bytes
 // for dims 1.., box in elements.  Out-of-range elements of a box read as zero.
 bool make_map(CUtensorMap *m, int rank, const void *ptr, const cuuint64_t *dims,
-              const cuuint64_t *strides, const cuuint32_t *box) {
+              const cuuint64_t *strides, const cuuint32_t *box,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(ptr), dims,
+    return fn(m, dtype, (cuuint32_t)rank, const_cast<void *>(ptr), dims,
               strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -70,7 +71,8 @@ int sm_count() {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int BN, int CG>
-GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &args,
+GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tc,
+               const GemmArgs &args,
                cudaStream_t st) {
     using Cfg = GemmCfg<BN, CG>;
     static bool attr_done[64] = {};
@@ -87,30 +89,31 @@ GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &arg
     const int tiles = args.num_m_tiles * args.num_n_tiles;
     const int groups = std::min(tiles, sm_count() / CG);
     const cudaError_t e = launch_pdl(gemm_tc_kernel<BN, CG>, dim3(groups * CG), dim3(kGemmThreads),
-                                     Cfg::SMEM_BYTES, st, CG, ta, tb, args);
+                                     Cfg::SMEM_BYTES, st, CG, ta, tb, tc, args);
     return e == cudaSuccess ? GemmStatus::kOk : GemmStatus::kLaunch;
 }
 
 GemmStatus dispatch(int bn, int cg, const CUtensorMap &ta, const CUtensorMap &tb,
+                    const CUtensorMap &tc,
                     const GemmArgs &args, cudaStream_t st) {
     if (cg == 2) {
         switch (bn) {
-            case 64: return run<64, 2>(ta, tb, args, st);
-            case 128: return run<128, 2>(ta, tb, args, st);
-            case 192: return run<192, 2>(ta, tb, args, st);
-            case 240: return run<240, 2>(ta, tb, args, st);
-            case 256: return run<256, 2>(ta, tb, args, st);
+            case 64: return run<64, 2>(ta, tb, tc, args, st);
+            case 128: return run<128, 2>(ta, tb, tc, args, st);
+            case 192: return run<192, 2>(ta, tb, tc, args, st);
+            case 240: return run<240, 2>(ta, tb, tc, args, st);
+            case 256: return run<256, 2>(ta, tb, tc, args, st);
             default: return GemmStatus::kBadShape;
         }
     }
     switch (bn) {
-        case 16: return run<16, 1>(ta, tb, args, st);
-        case 32: return run<32, 1>(ta, tb, args, st);
-        case 64: return run<64, 1>(ta, tb, args, st);
-        case 128: return run<128, 1>(ta, tb, args, st);
-        case 192: return run<192, 1>(ta, tb, args, st);
-        case 240: return run<240, 1>(ta, tb, args, st);
-        case 256: return run<256, 1>(ta, tb, args, st);
+        case 16: return run<16, 1>(ta, tb, tc, args, st);
+        case 32: return run<32, 1>(ta, tb, tc, args, st);
+        case 64: return run<64, 1>(ta, tb, tc, args, st);
+        case 128: return run<128, 1>(ta, tb, tc, args, st);
+        case 192: return run<192, 1>(ta, tb, tc, args, st);
+        case 240: return run<240, 1>(ta, tb, tc, args, st);
+        case 256: return run<256, 1>(ta, tb, tc, args, st);
         default: return GemmStatus::kBadShape;
     }
 }
@@ -184,7 +187,23 @@ GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
     args.status = L.status;
     args.timeout_ns = L.timeout_ns;
     args.fault_inject = L.fault_inject;
-    return dispatch(bn, cg, ta, tb, args, st);
+    // Row-major outputs whose per-warp column range (bn / 2) is a whole number
+    // of 128-byte pieces leave through shared memory and TMA stores.
+    CUtensorMap tc = tb;  // unused unless tma_out
+    const bool f32 = L.epi == kEpiResidF32 || L.epi == kEpiF32;
+    const bool row_major = f32 || L.epi == kEpiBf16 || L.epi == kEpiBf16Gelu;
+    const int pcols = f32 ? 32 : 64;
+    if (row_major && (bn / 2) % pcols == 0 && L.ldo >= L.N) {
+        const size_t es = f32 ? 4 : 2;
+        const cuuint64_t dc[2] = {(cuuint64_t)L.N, (cuuint64_t)L.M};
+        const cuuint64_t sc[1] = {(cuuint64_t)L.ldo * es};
+        const cuuint32_t bc[2] = {(cuuint32_t)pcols, 32};
+        if (!make_map(&tc, 2, L.out, dc, sc, bc,
+                      f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+            return GemmStatus::kTensorMap;
+        args.tma_out = 1;
+    }
+    return dispatch(bn, cg, ta, tb, tc, args, st);
 }
 
 GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
@@ -227,7 +246,7 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     args.dst_cols = L.dst_cols;
     args.status = L.status;
     args.timeout_ns = L.timeout_ns;
-    return dispatch(bn, cg, ta, tb, args, st);
+    return dispatch(bn, cg, ta, tb, tb, args, st);  // no TMA-store epilogue
 }
 
 }  // namespace aut

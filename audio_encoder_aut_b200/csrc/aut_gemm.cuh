@@ -60,6 +60,10 @@ struct GemmArgs {
     int *status;
     unsigned long long timeout_ns;
     int fault_inject;
+    // Epilogue stores through shared memory and TMA (tmC): plain row-major
+    // outputs (kEpiBf16, kEpiBf16Gelu, kEpiResidF32, kEpiF32) whose per-warp
+    // column range is a whole number of 128-byte pieces.
+    int tma_out;
 };
 
 // BN: tile width of one MMA (N).  CG: CTAs per MMA (1, or 2 for a CTA pair
@@ -78,8 +82,12 @@ struct GemmCfg {
                                      : (2 * BN <= 128) ? 128
                                      : (2 * BN <= 256) ? 256
                                                        : 512;
+    // Output staging for the TMA-store epilogue: 32 rows x 128 bytes per
+    // epilogue warp (one 128-byte-swizzled box).
+    static constexpr int STAGING_BYTES = 8 * 4096;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + BAR_BYTES;
+    static constexpr int SMEM_BYTES =
+        1024 /*alignment slack*/ + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
     static_assert(B_ROWS % 8 == 0, "each CTA holds whole 8-row swizzle atoms of B");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay aligned");
@@ -131,7 +139,7 @@ AUT_DEV void add_bias16(float (&v)[16], const __nv_bfloat16 *bias, int n0) {
 template <int BN, int CG>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
     using Cfg = GemmCfg<BN, CG>;
     constexpr int STAGES = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -139,7 +147,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * Cfg::A_BYTES;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * Cfg::STAGE_BYTES);
+    uint8_t *staging = smem + STAGES * Cfg::STAGE_BYTES;  // 1024-aligned: whole stages before it
+    uint64_t *full = reinterpret_cast<uint64_t *>(staging + Cfg::STAGING_BYTES);
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
@@ -273,7 +282,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t idesc =
                 args.f16 ? idesc_f16_f32(128 * CG, BN) : idesc_bf16_f32(128 * CG, BN);
             constexpr uint16_t kPair = 0x3;
-            const bool resid_mode = args.epi == kEpiResidF32;
+            // Residual preloaded into the accumulator the MMAs add onto, unless
+            // every CTA has a single tile: then the residual waits in the other
+            // accumulator and the MMAs start at once.
+            const bool resid_mode =
+                args.epi == kEpiResidF32 && !(args.tma_out && total_tiles <= n_groups);
             int stage = 0, it = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -343,6 +356,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int r = quad * 32 + lane;
         constexpr int NC = BN / 16;
         const bool resid = args.epi == kEpiResidF32;
+        // Single tile per CTA: the residual (x + bias) goes to accumulator 1
+        // while the MMAs fill accumulator 0; the drain adds the two.
+        const bool resid_once = resid && args.tma_out && total_tiles <= n_groups;
         bool ok = true;
         const uint32_t tempty_even = CG == 2 ? map_to_rank(tempty, 0) : 0;
         auto release = [&](int acc) {  // accumulator `acc` may be (re)written by the MMAs
@@ -399,7 +415,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         };
         // Residual mode: accumulator `acc` <- x + bias over this thread's row and chunks.
-        auto preload = [&](int tile, int acc) {
+        auto preload = [&](int tile, int acc, bool rel) {
             bool valid;
             size_t dst_row;
             int pos_row;
@@ -407,13 +423,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int n_base = (tile % args.num_n_tiles) * BN;
             const float *xp = reinterpret_cast<const float *>(args.out) + dst_row + n_base;
             const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+            // The chunks this warp drains (so that it only ever overwrites what it
+            // has itself drained, and reads back only what it has itself written):
+            // a contiguous half of the columns for the TMA drain, else alternate
+            // 16-column chunks.
+            const int c_first = args.tma_out ? half * (NC / 2) : half;
+            const int c_step = args.tma_out ? 1 : 2;
+            const int c_count = args.tma_out ? NC / 2 : (NC - half + 1) / 2;
 #pragma unroll 1
-            for (int c0 = half; c0 < NC; c0 += 8) {  // four chunks of loads in flight
+            for (int i0 = 0; i0 < c_count; i0 += 4) {  // four chunks of loads in flight
                 float v[4][16];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + 2 * u;
-                    if (c < NC) {
+                    const int c = c_first + (i0 + u) * c_step;
+                    if (i0 + u < c_count) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const float4 e = valid ? reinterpret_cast<const float4 *>(xp + c * 16)[q]
@@ -427,25 +450,109 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + 2 * u;
-                    if (c < NC) {
+                    const int c = c_first + (i0 + u) * c_step;
+                    if (i0 + u < c_count) {
                         add_bias16(v[u], args.bias, n_base + c * 16);
                         tmem_st16(t_addr + c * 16, v[u]);
                     }
                 }
             }
             tc_wait_st();
-            release(acc);
+            if (rel) release(acc);
         };
 
-        if (resid) {  // the first two accumulators start from the residual
+        // Drain through shared memory: this warp's 32 rows x BN / 2 columns go
+        // out in pieces of 32 rows x 128 bytes (32 fp32 or 64 bf16 columns),
+        // each written to the warp's 128-byte-swizzled staging box and stored
+        // by one TMA tile store (whole lines, rows past M clipped by the map).
+        auto drain_tma = [&](int tile, uint32_t t_acc) {
+            constexpr int HW = BN / 2;
+            const bool f32 = args.epi == kEpiResidF32 || args.epi == kEpiF32;
+            const int pcols = f32 ? 32 : 64;
+            uint8_t *stg = staging + (warp - 2) * 4096;
+            const int m0 = ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32;
+            const bool slab = m0 < args.M;  // warp-uniform
+            const int n_first = (tile % args.num_n_tiles) * BN + half * HW;
+            const uint32_t t_res = tmem_base + ((uint32_t)(quad * 32) << 16) + BN + half * HW;
+            t_acc += half * HW;
+#pragma unroll 1
+            for (int p = 0; p < HW / pcols; ++p) {
+                uint32_t w[32];  // this row's 128-byte piece as 8 chunks of 4 words
+                if (f32) {
+                    float v[2][16];
+                    tmem_ld16(t_acc + p * pcols, v[0]);
+                    tmem_ld16(t_acc + p * pcols + 16, v[1]);
+                    if (resid_once) {
+                        float r[2][16];
+                        tmem_ld16(t_res + p * pcols, r[0]);
+                        tmem_ld16(t_res + p * pcols + 16, r[1]);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) v[i][j] += r[i][j];
+                    } else {
+                        tc_wait_ld();
+                        if (!resid) {
+                            add_bias16(v[0], args.bias, n_first + p * pcols);
+                            add_bias16(v[1], args.bias, n_first + p * pcols + 16);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j >> 4][j & 15]);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {  // 32 columns at a time
+                        float v[2][16];
+                        tmem_ld16(t_acc + p * pcols + 32 * h, v[0]);
+                        tmem_ld16(t_acc + p * pcols + 32 * h + 16, v[1]);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            add_bias16(v[i], args.bias, n_first + p * pcols + 32 * h + 16 * i);
+                            if (args.epi == kEpiBf16Gelu) {
+#pragma unroll
+                                for (int j = 0; j < 16; j += 2) {
+                                    const float2 g = gelu_fast2(make_float2(v[i][j], v[i][j + 1]));
+                                    v[i][j] = g.x;
+                                    v[i][j + 1] = g.y;
+                                }
+                            }
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                w[16 * h + 8 * i + j] = pack_bf16x2(v[i][2 * j], v[i][2 * j + 1]);
+                        }
+                    }
+                }
+                // The previous piece's store has finished reading the box.
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+                uint8_t *row = stg + lane * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)  // 16-byte chunk j of this row, 128-byte swizzle
+                    *reinterpret_cast<uint4 *>(row + ((j ^ (lane & 7)) << 4)) =
+                        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && slab) {
+                    tma_store_2d(&tmC, stg, n_first + p * pcols, m0);
+                    bulk_commit();
+                }
+            }
+        };
+
+        if (resid_once) {
+            if (group < total_tiles) preload(group, 1, false);
+        } else if (resid) {  // the first two accumulators start from the residual
             int t = group;
-            for (int a = 0; a < 2 && t < total_tiles; ++a, t += n_groups) preload(t, a);
+            for (int a = 0; a < 2 && t < total_tiles; ++a, t += n_groups) preload(t, a, true);
         }
         int it = 0;
         for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
+            if (args.tma_out && args.bias && !resid && lane * 4 < BN / 2)  // warm L1 with the bias
+                prefetch_l1(args.bias + (tile % args.num_n_tiles) * BN + half * (BN / 2) + lane * 4);
             if (!mbar_wait(tfull + acc, acc_phase, abort_v, lim)) {
                 ok = false;
                 break;
@@ -457,6 +564,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int pos_row;
             locate(tile, valid, dst_row, pos_row);
             const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+            if (args.tma_out) {
+                drain_tma(tile, t_addr);
+            } else {
 #pragma unroll 1
             for (int c0 = half; c0 < NC; c0 += 4) {
                 const int c1 = c0 + 2;
@@ -532,17 +642,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             }
+            }
             if (resid) {
                 const int next = tile + 2 * n_groups;  // the tile this accumulator serves next
                 if (next < total_tiles) {
                     tc_fence_before();  // finish reading the drained values before rewriting
-                    preload(next, acc);
+                    preload(next, acc, true);
                 }
             } else {
                 release(acc);
             }
         }
         if (!ok && lane == 0) gemm_signal_abort(args, abort_v);
+        if (args.tma_out && lane == 0) bulk_wait_all();  // stores complete before exit
+        __syncwarp();
     }
 
     __syncwarp();

@@ -29,7 +29,10 @@ def _rand(shape, seed, scale=1.0):
 
 SHAPES = [(1, 64, 64), (31, 192, 64), (128, 256, 256), (300, 1280, 1280), (1000, 3840, 1280),
           (257, 2688, 896), (390, 3584, 896), (77, 16, 64), (129, 240, 7680), (4000, 5120, 1280),
-          (3000, 1280, 5120), (513, 2048, 1280), (45, 1024, 896)]
+          (3000, 1280, 5120), (513, 2048, 1280), (45, 1024, 896),
+          # K = 64: one k-block per tile, so a CTA drains one tile while it
+          # preloads the residual of its next - the two must not overlap columns
+          (8192, 1280, 64), (2000, 512, 64)]
 
 
 @pytest.mark.parametrize("flags", [0, A.LINEAR_SINGLE_CTA], ids=["auto", "single_cta"])
