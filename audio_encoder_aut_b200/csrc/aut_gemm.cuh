@@ -83,8 +83,10 @@ struct GemmCfg {
                                      : (2 * BN <= 256) ? 256
                                                        : 512;
     // Output staging for the TMA-store epilogue: 32 rows x 128 bytes per
-    // epilogue warp (one 128-byte-swizzled box).
-    static constexpr int STAGING_BYTES = 8 * 4096;
+    // epilogue warp (one 128-byte-swizzled box), for tile widths whose half is
+    // a whole number of 32-column fp32 pieces (no other width can use it, and
+    // shared memory left unallocated serves as L1 cache).
+    static constexpr int STAGING_BYTES = (BN / 2) % 32 == 0 ? 8 * 4096 : 0;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES =
         1024 /*alignment slack*/ + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
@@ -193,7 +195,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     else
         __syncthreads();
     tc_fence_after();
-    pdl_wait();  // the previous kernel's outputs (this GEMM's A, residual) are complete
     const uint32_t tmem_base = *tmem_slot;
     volatile int *abort_v = abort_flag;
     const int total_tiles = args.num_m_tiles * args.num_n_tiles;
@@ -205,6 +206,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // Both CTAs of a pair load their own A rows and B half; the loads of
             // both complete on the even CTA's `full` barrier, which the even CTA
             // arms with the pair's byte count.
+            const uint32_t a_bytes =
+                args.conv ? 128u * args.conv_rows * args.conv_cols : (uint32_t)Cfg::A_BYTES;
+            auto arm = [&](int stage) {
+                if (rank == 0) mbar_arrive_expect_tx(full + stage, CG * (a_bytes + Cfg::B_BYTES));
+            };
+            // Weights (B): k-block kb of the tile whose B rows start at b_row.
+            auto load_b = [&](int stage, int kb, int b_row) {
+                uint8_t *b_dst = sB + stage * Cfg::B_BYTES;
+                if (!args.conv) {
+                    if constexpr (CG == 2)
+                        tma_load_2d_pair(b_dst, &tmB, map_to_rank(full + stage, 0), kb * 64, b_row);
+                    else
+                        tma_load_2d(b_dst, &tmB, full + stage, kb * 64, b_row);
+                } else {
+                    const int tap = kb / args.conv_cblocks;
+                    const int cb = kb - tap * args.conv_cblocks;
+                    if constexpr (CG == 2)
+                        tma_load_3d_pair(b_dst, &tmB, map_to_rank(full + stage, 0), cb * 64, tap,
+                                         b_row);
+                    else
+                        tma_load_3d(b_dst, &tmB, full + stage, cb * 64, tap, b_row);
+                }
+            };
+            // Activations (A): k-block kb of the tile at 128-row slot m_slot.
+            auto load_a = [&](int stage, int kb, int m_slot) {
+                uint8_t *a_dst = sA + stage * Cfg::A_BYTES;
+                if (!args.conv) {
+                    if constexpr (CG == 2)
+                        tma_load_2d_pair(a_dst, &tmA, map_to_rank(full + stage, 0), kb * 64,
+                                         m_slot * 128);
+                    else
+                        tma_load_2d(a_dst, &tmA, full + stage, kb * 64, m_slot * 128);
+                } else {
+                    const int tap = kb / args.conv_cblocks;
+                    const int cb = kb - tap * args.conv_cblocks;
+                    const int kh = tap / 3, kw = tap - 3 * (tap / 3);
+                    // tap kh reads input row 2i + kh - 1: phase 1 for kh in {0, 2},
+                    // phase 0 for kh = 1; plane row i (kh = 0) or i + 1 (kh = 1, 2)
+                    // counting the leading zero row.  Same for kw along columns.
+                    const int plane = (kh == 1 ? 0 : 2) + (kw == 1 ? 0 : 1);
+                    const int dh = kh == 0 ? 0 : 1, dw = kw == 0 ? 0 : 1;
+                    const int vrow = m_slot * args.conv_rows + dh;
+                    if constexpr (CG == 2)
+                        tma_load_4d_pair(a_dst, &tmA, map_to_rank(full + stage, 0), cb * 64, dw,
+                                         vrow, plane);
+                    else
+                        tma_load_4d(a_dst, &tmA, full + stage, cb * 64, dw, vrow, plane);
+                }
+            };
+            pdl_wait();  // the previous kernel's outputs (this GEMM's A) are complete
             int stage = 0;
             uint32_t phase = 0, issued = 0, parity = 0;
             bool ok = true, skip = args.fault_inject != 0 && blockIdx.x == 0;
@@ -220,40 +271,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (skip) {
                         skip = false;  // injected fault: this stage is never filled
                     } else {
-                        uint8_t *a_dst = sA + stage * Cfg::A_BYTES;
-                        uint8_t *b_dst = sB + stage * Cfg::B_BYTES;
-                        const uint32_t a_bytes =
-                            args.conv ? 128u * args.conv_rows * args.conv_cols : (uint32_t)Cfg::A_BYTES;
-                        if (rank == 0)
-                            mbar_arrive_expect_tx(full + stage, CG * (a_bytes + Cfg::B_BYTES));
-                        if (!args.conv) {
-                            if constexpr (CG == 2) {
-                                const uint32_t bar = map_to_rank(full + stage, 0);
-                                tma_load_2d_pair(a_dst, &tmA, bar, kb * 64, m_slot * 128);
-                                tma_load_2d_pair(b_dst, &tmB, bar, kb * 64, b_row);
-                            } else {
-                                tma_load_2d(a_dst, &tmA, full + stage, kb * 64, m_slot * 128);
-                                tma_load_2d(b_dst, &tmB, full + stage, kb * 64, b_row);
-                            }
-                        } else {
-                            const int tap = kb / args.conv_cblocks;
-                            const int cb = kb - tap * args.conv_cblocks;
-                            const int kh = tap / 3, kw = tap - 3 * (tap / 3);
-                            // tap kh reads input row 2i + kh - 1: phase 1 for kh in {0, 2},
-                            // phase 0 for kh = 1; plane row i (kh = 0) or i + 1 (kh = 1, 2)
-                            // counting the leading zero row.  Same for kw along columns.
-                            const int plane = (kh == 1 ? 0 : 2) + (kw == 1 ? 0 : 1);
-                            const int dh = kh == 0 ? 0 : 1, dw = kw == 0 ? 0 : 1;
-                            const int vrow = m_slot * args.conv_rows + dh;
-                            if constexpr (CG == 2) {
-                                const uint32_t bar = map_to_rank(full + stage, 0);
-                                tma_load_4d_pair(a_dst, &tmA, bar, cb * 64, dw, vrow, plane);
-                                tma_load_3d_pair(b_dst, &tmB, bar, cb * 64, tap, b_row);
-                            } else {
-                                tma_load_4d(a_dst, &tmA, full + stage, cb * 64, dw, vrow, plane);
-                                tma_load_3d(b_dst, &tmB, full + stage, cb * 64, tap, b_row);
-                            }
-                        }
+                        arm(stage);
+                        load_b(stage, kb, b_row);
+                        load_a(stage, kb, m_slot);
                         issued |= 1u << stage;
                         parity = (parity & ~(1u << stage)) | (phase << stage);
                     }
@@ -351,6 +371,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // Residual mode: the accumulator is pre-loaded with x + bias (tcgen05.st)
         // while the MMAs run on the other accumulator, the MMAs add onto it, and
         // draining is a plain store - no load sits on the tile's critical path.
+        pdl_wait();  // the residual and the output buffers belong to the previous kernel
         const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
         const int half = (warp - 2) >> 2;
         const int r = quad * 32 + lane;

@@ -261,20 +261,37 @@ AUT_DEV uint32_t pack_f16x2_sat(float a, float b) {
 AUT_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 AUT_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// GELU(x) = x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2 (the exact form), with erf
-// from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.25:
-// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3) exp(-z^2), t = 1 / (1 + p z), z >= 0,
-// |error| <= 2.5e-5 (two orders below the bf16 rounding of the results);
-// odd symmetry for z < 0.
-constexpr float kErfP = 0.47047f, kErfA1 = 0.3480242f, kErfA2 = -0.0958798f,
-                kErfA3 = 0.7478556f;
+// GELU(x) = x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2, the exact form, with one
+// exp2 per value.  For a = min(|x|, 6):
+//   Phi(-a) = exp2(S(a) - a^2 log2(e) / 2),
+// where S is a degree-10 polynomial least-squares fitted to
+// log2 Phi(-a) + a^2 log2(e) / 2 on [0, 6] (gen_gelu_poly.py beside this file
+// regenerates the coefficients).  Evaluated in fp32 the GELU is off by at most
+// 7e-8 in absolute terms; Phi(-6) ~ 1e-9 bounds what the clamp leaves out.
+// Then GELU(x) = x (1 - Phi(-a)) for x >= 0 and x Phi(-a) for x < 0.
+constexpr float kHalfLog2e = 0.72134752044448170f;  // log2(e) / 2
+
+AUT_DEV float ex2_approx(float t) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(t));
+    return r;
+}
 
 AUT_DEV float gelu_fast(float x) {
-    const float z = fabsf(x) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(kErfP, z, 1.0f));
-    const float poly = fmaf(fmaf(kErfA3, t, kErfA2), t, kErfA1) * t;
-    const float erf_abs = fmaf(-poly, __expf(-z * z), 1.0f);
-    return 0.5f * x * (1.0f + copysignf(erf_abs, x));
+    const float a = fminf(fabsf(x), 6.0f);
+    float s = -1.149771656e-08f;
+    s = fmaf(s, a, 3.877935626e-07f);
+    s = fmaf(s, a, -5.562640126e-06f);
+    s = fmaf(s, a, 4.234902372e-05f);
+    s = fmaf(s, a, -1.503860694e-04f);
+    s = fmaf(s, a, -3.018761636e-04f);
+    s = fmaf(s, a, 7.375840098e-03f);
+    s = fmaf(s, a, -5.279456079e-02f);
+    s = fmaf(s, a, 2.622790337e-01f);
+    s = fmaf(s, a, -1.151131988e+00f);
+    s = fmaf(s, a, -9.999987483e-01f);
+    const float h = ex2_approx(fmaf(-kHalfLog2e * a, a, s));  // Phi(-a)
+    return x * (x >= 0.0f ? 1.0f - h : h);
 }
 
 // Packed fp32x2 arithmetic (two lanes per instruction).
@@ -293,17 +310,21 @@ AUT_DEV float2 fmul2(float2 a, float2 b) {
 
 // gelu_fast on two values, the polynomial and scaling in packed fp32x2.
 AUT_DEV float2 gelu_fast2(float2 x) {
-    const float2 z = make_float2(fabsf(x.x) * 0.70710678118654752f, fabsf(x.y) * 0.70710678118654752f);
-    const float2 den = ffma2(make_float2(kErfP, kErfP), z, make_float2(1.f, 1.f));
-    const float2 t = make_float2(__fdividef(1.0f, den.x), __fdividef(1.0f, den.y));
-    float2 poly = ffma2(make_float2(kErfA3, kErfA3), t, make_float2(kErfA2, kErfA2));
-    poly = ffma2(poly, t, make_float2(kErfA1, kErfA1));
-    poly = fmul2(poly, t);
-    const float2 zz = fmul2(z, z);
-    const float2 e = make_float2(__expf(-zz.x), __expf(-zz.y));
-    const float2 erf_abs = ffma2(make_float2(-poly.x, -poly.y), e, make_float2(1.f, 1.f));
-    const float2 one_plus = make_float2(1.0f + copysignf(erf_abs.x, x.x), 1.0f + copysignf(erf_abs.y, x.y));
-    return fmul2(fmul2(make_float2(0.5f, 0.5f), x), one_plus);
+    const float2 a = make_float2(fminf(fabsf(x.x), 6.0f), fminf(fabsf(x.y), 6.0f));
+    float2 s = make_float2(-1.149771656e-08f, -1.149771656e-08f);
+    s = ffma2(s, a, make_float2(3.877935626e-07f, 3.877935626e-07f));
+    s = ffma2(s, a, make_float2(-5.562640126e-06f, -5.562640126e-06f));
+    s = ffma2(s, a, make_float2(4.234902372e-05f, 4.234902372e-05f));
+    s = ffma2(s, a, make_float2(-1.503860694e-04f, -1.503860694e-04f));
+    s = ffma2(s, a, make_float2(-3.018761636e-04f, -3.018761636e-04f));
+    s = ffma2(s, a, make_float2(7.375840098e-03f, 7.375840098e-03f));
+    s = ffma2(s, a, make_float2(-5.279456079e-02f, -5.279456079e-02f));
+    s = ffma2(s, a, make_float2(2.622790337e-01f, 2.622790337e-01f));
+    s = ffma2(s, a, make_float2(-1.151131988e+00f, -1.151131988e+00f));
+    s = ffma2(s, a, make_float2(-9.999987483e-01f, -9.999987483e-01f));
+    const float2 t = ffma2(fmul2(make_float2(-kHalfLog2e, -kHalfLog2e), a), a, s);
+    const float h0 = ex2_approx(t.x), h1 = ex2_approx(t.y);  // Phi(-a)
+    return fmul2(x, make_float2(x.x >= 0.0f ? 1.0f - h0 : h0, x.y >= 0.0f ? 1.0f - h1 : h1));
 }
 
 AUT_DEV uint32_t pack_bf16x2(float a, float b) {
