@@ -20,7 +20,7 @@
 //              the O product of tile k - 1
 //   warps 2-9  softmax and epilogue, two warps per TMEM lane quadrant, each
 //              over half of the keys: row max (exchanged between the two
-//              halves), p = exp2((s - max) * log2(e) / sqrt(64)) written to
+//              halves), p = exp2(s log2(e) / sqrt(64) - max log2(e) / sqrt(64)) written to
 //              shared memory as fp16 (P lies in [0, 1]; fp16 keeps 11
 //              significant bits, 8x finer than bf16) in the swizzled K-major
 //              layout the MMA reads, over the Q and K tiles the first MMA no
@@ -198,29 +198,44 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
             // -------------------------------------------------- MMA issuer --
             constexpr uint32_t idesc_o = idesc_f16_f32_bmn(kTile, kHd);
             bool ok = true;
+            // S of local tile kk (global tile t): N = the window's keys rounded up
+            // to 16.  Needs the tile's loads and a free S buffer.
+            auto issue_s = [&](int kk, int t) -> bool {
+                int s0, len, n16;
+                window_of(cu, t / heads, &s0, &len, &n16);
+                const int s = kk % kStages;
+                if (!mbar_wait(full + s, (uint32_t)(kk / kStages) & 1u, abort_v, kTimeoutNs))
+                    return false;
+                tc_fence_after();
+                uint8_t *st = sm + s * kStageBytes;
+                const uint32_t idesc_s = idesc_bf16_f32(kTile, 16 * n16);
+#pragma unroll
+                for (int q = 0; q < kHd / 16; ++q)
+                    tc_mma_bf16(tmem, smem_desc_sw128(st) + 2 * q,
+                                smem_desc_sw128(st + kTileBytes) + 2 * q, idesc_s, q > 0);
+                tc_commit(s_full);
+                return true;
+            };
             int k = 0;
+            if (blockIdx.x < n_tiles) ok = issue_s(0, blockIdx.x);
             for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++k) {
                 int s0, len, n16;
                 window_of(cu, t / heads, &s0, &len, &n16);
                 const int s = k % kStages;
-                const uint32_t use = (uint32_t)(k / kStages);
                 uint8_t *st = sm + s * kStageBytes;
-                if (!mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs)) {
+                // P of tile k is in shared memory and S has been read: S of the
+                // next tile goes first (the softmax waits for it), then O of this.
+                if (!mbar_wait(p_full, k & 1u, abort_v, kTimeoutNs)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                // S over the window's keys only (N = 16 n16 columns).
-                const uint32_t idesc_s = idesc_bf16_f32(kTile, 16 * n16);
-#pragma unroll
-                for (int kk = 0; kk < kHd / 16; ++kk)
-                    tc_mma_bf16(tmem, smem_desc_sw128(st) + 2 * kk,
-                                smem_desc_sw128(st + kTileBytes) + 2 * kk, idesc_s, kk > 0);
-                tc_commit(s_full);
+                if (t + (int)gridDim.x < n_tiles && !issue_s(k + 1, t + gridDim.x)) {
+                    ok = false;
+                    break;
+                }
                 // O buffer k & 1 was last drained by the epilogue of tile k - 2.
                 const int ob = k & 1;
-                if (!mbar_wait(p_full, k & 1u, abort_v, kTimeoutNs) ||
-                    (k >= 2 && !mbar_wait(o_empty + ob, ((k - 2) >> 1) & 1u, abort_v, kTimeoutNs))) {
+                if (k >= 2 && !mbar_wait(o_empty + ob, ((k - 2) >> 1) & 1u, abort_v, kTimeoutNs)) {
                     ok = false;
                     break;
                 }
@@ -294,21 +309,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
             const bool active = quad * 32 < len;  // warp-uniform: some rows are valid
             fail = fail || !mbar_wait(s_full, k & 1u, abort_v, kTimeoutNs);
             fail = __any_sync(0xffffffffu, fail);
+            // This warp's scores: keys 64 half .. 64 half + 64.
             float mx = -INFINITY;
+            const int kbase = half * 64;
             if (!fail) {
                 tc_fence_after();
-                // Row max over this warp's half of the keys.
                 if (active) {
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
-                        const int key0 = half * 64 + c * 32;
+                        const int key0 = kbase + c * 32;
                         if (key0 < len) {  // uniform: the block shares `len`
                             float v[32];
                             tmem_ld32(trow + key0, v);
                             tc_wait_ld();
+                            if (key0 + 32 <= len) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (key0 + j < len) mx = fmaxf(mx, v[j]);
+                                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
+                            } else {  // the chunk holding the window's end
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (key0 + j < len) mx = fmaxf(mx, v[j]);
+                            }
                         }
                     }
                 }
@@ -319,15 +340,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
                 break;
             }
             mx = fmaxf(red_max[row], red_max[kTile + row]);
-            // P = exp of the scaled, shifted scores; zero past the window's end.
+            // P = exp2(s * scale - max * scale); zero past the window's end.
+            const float neg = -mx * scale_log2e;
             float sum = 0.f;
             if (active) {
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    const int key0 = half * 64 + c * 32;
+                    const int key0 = kbase + c * 32;
                     if (key0 < len) {
-                        float v[32];
-                        tmem_ld32(trow + key0, v);
+                        const bool whole = key0 + 32 <= len;
+                        float v[1][32];
+                        tmem_ld32(trow + key0, v[0]);
                         tc_wait_ld();
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {  // 8 keys = one 16-byte chunk of P
@@ -335,10 +358,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int j = q * 8 + 2 * e;
-                                const float p0 =
-                                    key0 + j < len ? exp2f((v[j] - mx) * scale_log2e) : 0.f;
-                                const float p1 =
-                                    key0 + j + 1 < len ? exp2f((v[j + 1] - mx) * scale_log2e) : 0.f;
+                                float p0 = ex2_approx(fmaf(v[0][j], scale_log2e, neg));
+                                float p1 = ex2_approx(fmaf(v[0][j + 1], scale_log2e, neg));
+                                if (!whole) {
+                                    p0 = key0 + j < len ? p0 : 0.f;
+                                    p1 = key0 + j + 1 < len ? p1 : 0.f;
+                                }
                                 sum += p0 + p1;
                                 __half2 hp = __floats2half2_rn(p0, p1);
                                 ph[e] = *reinterpret_cast<uint32_t *>(&hp);

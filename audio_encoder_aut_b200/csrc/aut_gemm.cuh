@@ -155,7 +155,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
     uint64_t *mma_done = tempty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *xbar = mma_done + 1;  // [8] per epilogue warp: residual piece landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xbar + kEpilogueWarps);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     pdl_trigger();
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(tempty + a, kEpilogueWarps * CG);
         }
         mbar_init(mma_done, 1);
+        for (int w = 0; w < kEpilogueWarps; ++w) mbar_init(xbar + w, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -302,11 +304,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t idesc =
                 args.f16 ? idesc_f16_f32(128 * CG, BN) : idesc_bf16_f32(128 * CG, BN);
             constexpr uint16_t kPair = 0x3;
-            // Residual preloaded into the accumulator the MMAs add onto, unless
-            // every CTA has a single tile: then the residual waits in the other
-            // accumulator and the MMAs start at once.
-            const bool resid_mode =
-                args.epi == kEpiResidF32 && !(args.tma_out && total_tiles <= n_groups);
+            // Residual preloaded into the accumulator the MMAs add onto on the
+            // per-row store path; with the TMA-store drain the MMAs start from
+            // zero and the drain adds the residual.
+            const bool resid_mode = args.epi == kEpiResidF32 && !args.tma_out;
             int stage = 0, it = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -331,8 +332,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tc_fence_after();
                     const uint64_t a_desc = smem_desc_sw128(sA + stage * Cfg::A_BYTES);
                     const uint64_t b_desc = smem_desc_sw128(sB + stage * Cfg::B_BYTES);
+                    // A convolution's last channel block of each tap may be partly
+                    // past C (zero fill): only its K steps that hold channels run.
+                    int ksteps = 4;
+                    if (args.conv) {
+                        const int cb = kb % args.conv_cblocks;
+                        const int left = args.C - cb * 64;
+                        if (left < 64) ksteps = (left + 15) >> 4;
+                    }
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {  // K = 16 per MMA: +32 bytes in the row
+                        if (kk >= ksteps) break;
                         const uint32_t accumulate = resid_mode || (kb | kk) != 0;
                         if constexpr (CG == 2)
                             tc_mma_bf16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
@@ -380,6 +390,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // Single tile per CTA: the residual (x + bias) goes to accumulator 1
         // while the MMAs fill accumulator 0; the drain adds the two.
         const bool resid_once = resid && args.tma_out && total_tiles <= n_groups;
+        // Several tiles per CTA: the drain brings each residual piece in by TMA
+        // (into the staging box it then stores from) and adds it there.
+        const bool resid_drain = resid && args.tma_out && !resid_once;
+        uint64_t *my_xbar = xbar + (warp - 2);
+        uint32_t xph = 0;        // phase of my_xbar
+        bool x_pending = false;  // lane 0: a residual load has not been waited for
+        // Residual piece (32 rows x 32 fp32) of `tile` at column offset `col`
+        // into this warp's staging box; lane 0 only.
+        auto load_x = [&](int tile, int col) {
+            const int m0 = ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32;
+            bulk_wait_read_all();  // the box's previous store has read it
+            mbar_arrive_expect_tx(my_xbar, 4096);
+            tma_load_2d(staging + (warp - 2) * 4096, &tmC, my_xbar,
+                        (tile % args.num_n_tiles) * BN + half * (BN / 2) + col, m0);
+            x_pending = true;
+        };
         bool ok = true;
         const uint32_t tempty_even = CG == 2 ? map_to_rank(tempty, 0) : 0;
         auto release = [&](int acc) {  // accumulator `acc` may be (re)written by the MMAs
@@ -513,10 +539,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                             for (int j = 0; j < 16; ++j) v[i][j] += r[i][j];
                     } else {
+                        if (resid_drain && slab && p > 0 && lane == 0) load_x(tile, p * pcols);
                         tc_wait_ld();
-                        if (!resid) {
+                        if (!resid || resid_drain) {
                             add_bias16(v[0], args.bias, n_first + p * pcols);
                             add_bias16(v[1], args.bias, n_first + p * pcols + 16);
+                        }
+                        if (resid_drain && slab) {  // + the residual piece from the box
+                            if (!mbar_wait(my_xbar, xph, abort_v, lim)) {
+                                ok = false;
+                                gemm_signal_abort(args, abort_v);
+                            } else {
+                                x_pending = false;
+                            }
+                            xph ^= 1u;
+                            const uint8_t *row = stg + lane * 128;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 x4 = *reinterpret_cast<const float4 *>(
+                                    row + ((j ^ (lane & 7)) << 4));
+                                float *q = &v[j >> 2][(j & 3) * 4];
+                                q[0] += x4.x;
+                                q[1] += x4.y;
+                                q[2] += x4.z;
+                                q[3] += x4.w;
+                            }
                         }
                     }
 #pragma unroll
@@ -564,7 +611,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
         if (resid_once) {
             if (group < total_tiles) preload(group, 1, false);
-        } else if (resid) {  // the first two accumulators start from the residual
+        } else if (resid && !args.tma_out) {  // the first two accumulators start from the residual
             int t = group;
             for (int a = 0; a < 2 && t < total_tiles; ++a, t += n_groups) preload(t, a, true);
         }
@@ -572,8 +619,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
-            if (args.tma_out && args.bias && !resid && lane * 4 < BN / 2)  // warm L1 with the bias
+            if (args.tma_out && args.bias && (!resid || resid_drain) && lane * 4 < BN / 2)
                 prefetch_l1(args.bias + (tile % args.num_n_tiles) * BN + half * (BN / 2) + lane * 4);
+            if (resid_drain && lane == 0 &&  // first residual piece lands during the mainloop
+                ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32 < args.M)
+                load_x(tile, 0);
             if (!mbar_wait(tfull + acc, acc_phase, abort_v, lim)) {
                 ok = false;
                 break;
@@ -664,7 +714,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
             }
-            if (resid) {
+            if (resid && !args.tma_out) {
                 const int next = tile + 2 * n_groups;  // the tile this accumulator serves next
                 if (next < total_tiles) {
                     tc_fence_before();  // finish reading the drained values before rewriting
@@ -676,6 +726,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok && lane == 0) gemm_signal_abort(args, abort_v);
         if (args.tma_out && lane == 0) bulk_wait_all();  // stores complete before exit
+        if (x_pending) mbar_wait(my_xbar, xph, nullptr, lim);  // a residual load in flight lands
         __syncwarp();
     }
 

@@ -64,6 +64,7 @@ WORKLOADS = {
     "asr06b_30s": ASR_06B,
     "omni_16req": OMNI,
     "omni_20min": OMNI,
+    "omni_20min_ragged": OMNI,
     "omni_256req": OMNI,
 }
 

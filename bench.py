@@ -355,6 +355,54 @@ def our_arm(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def sweep(args):
+    """Throughput against the packed total: Omni-class batches of requests with
+    log-uniform lengths on [0.5, 60] s, grown to each target token count; one
+    JSON line per point (CUDA-graph replay, L2 flushed between steps)."""
+    import numpy as np
+    import torch
+    from audio_encoder_aut_b200.encoder import Encoder
+
+    cfg = S.WORKLOADS["omni_256req"]
+    w = S.weights(cfg)
+    enc = Encoder(cfg, w, 0)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    pk = peaks()[0]
+    rng = np.random.default_rng(S.SEED_LENGTHS + 7)
+    pool = [int(round(100 * np.exp(rng.uniform(np.log(0.5), np.log(60.0))))) for _ in range(4096)]
+    for target in (1000, 2000, 5000, 10000, 20000, 50000, 100000, 200000):
+        lens, T = [], 0
+        while T < target:
+            lens.append(pool[len(lens)])
+            if sum(lens) * 0.13 >= target or len(lens) % 32 == 0:
+                T = enc.plan(lens)[2]
+        feats = S.features(lens, seed=S.SEED_FEATURES)
+        fd = enc.features_to_device(feats)
+        _, cu, T, nW, nch = enc.plan(lens)
+        out = torch.empty((T, cfg.output_dim), dtype=torch.float32, device="cuda")
+        graph, _ = enc.capture(fd, lens, out=out)
+        for _ in range(3):
+            graph.replay()
+        ms = []
+        for _ in range(5):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        t = sorted(ms)[len(ms) // 2]
+        flops = credited_flops(cfg, lens, cu)[0]
+        print(json.dumps({"sweep_tokens": T, "requests": len(lens), "audio_seconds": sum(lens) / 100,
+                          "ms_per_step": t, "audio_s_per_s": sum(lens) / 100 / (t / 1e3),
+                          "tokens_per_s": T / (t / 1e3), "tflops": flops / (t / 1e3) / 1e12,
+                          "pct_bf16_peak": 100 * flops / (t / 1e3) / 1e12 / pk}), flush=True)
+        del graph, out, fd
+    assert enc.check() == 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -366,7 +414,12 @@ def main():
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch the forward eagerly instead of replaying its CUDA graph")
     ap.add_argument("--cpu-sample-seconds", type=float, default=60.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the bench line, one line per packed total of 1k-200k tokens")
     args = ap.parse_args()
+    if args.sweep:
+        sweep(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     world = int(os.environ.get("WORLD_SIZE", "1"))
