@@ -3,7 +3,7 @@
 GELU(x) = x * Phi(x).  With a = min(|x|, 6):
     Phi(-a) = exp2(-a^2 * log2(e) / 2 + S(a)),
 and S(a) = log2(Phi(-a)) + a^2 * log2(e) / 2 is smooth on [0, 6].  S is fitted
-by Chebyshev least squares of degree 10 on a dense grid and converted to
+by Chebyshev least squares of degree 7 on a dense grid and converted to
 monomial coefficients for Horner evaluation in fp32.  Then
     GELU(x) = x * (1 - Phi(-a))  for x >= 0,   x * Phi(-a)  for x < 0,
 one exp2 per value.  The script prints the coefficients and the worst
@@ -13,7 +13,7 @@ Usage: python gen_gelu_poly.py
 import numpy as np
 from scipy.special import log_ndtr
 
-DEGREE, A_MAX = 10, 6.0
+DEGREE, A_MAX = 7, 6.0
 
 
 def fit():

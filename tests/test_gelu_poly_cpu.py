@@ -1,5 +1,5 @@
 """The device GELU's polynomial (aut_ptx.cuh, gelu_fast), evaluated here in
-fp32 as the kernels do, against the exact erf GELU x * Phi(x): within 1e-7
+fp32 as the kernels do, against the exact erf GELU x * Phi(x): within 5e-7
 plus the fp32 rounding of the result everywhere, including the clamped tails
 and x = 0."""
 import os
@@ -33,11 +33,11 @@ def _gelu_fp32(x):
 
 
 def test_device_gelu_polynomial_matches_exact_gelu():
-    assert len(_coefficients()) == 11
+    assert len(_coefficients()) == 8
     x = np.concatenate([np.linspace(-12, 12, 400001), [0.0, -6.0, 6.0, -1e-30, 1e-30]])
     ref = x * ndtr(x)
     err = np.abs(_gelu_fp32(x) - ref)
-    # fit error (<= 7e-8) plus the fp32 rounding of the final product and of 1 - h
-    bound = 1e-7 + 2.0 ** -22 * np.abs(ref)
+    # fit error (<= 4.8e-7) plus the fp32 rounding of the final product and of 1 - h
+    bound = 5e-7 + 2.0 ** -22 * np.abs(ref)
     assert (err <= bound).all(), (err - bound).max()
     assert _gelu_fp32(np.array([0.0]))[0] == 0.0
