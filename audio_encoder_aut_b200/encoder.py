@@ -152,6 +152,61 @@ class Encoder:
             self.encode(features, feature_lens, out=out, trace=trace)
         return graph, out
 
+    def encode_stream(self, host_features, feature_lens, host_outs, graphs=None,
+                      before_each=None):
+        """Encodes a sequence of batches of one shape from pinned host memory
+        into pinned host outputs: host_features[i] (bf16 [B, 128, T_max]) ->
+        host_outs[i] (fp32 [total_tokens, output_dim]).  Every batch is copied
+        in, encoded and copied back, and the copies of batches i + 1 and i - 1
+        run on a second stream while batch i computes (two device buffer sets,
+        each with its captured forward).  `graphs`, as returned by a previous
+        call, skips the captures; `before_each`, if given, is called on the
+        compute stream before every batch.  Returns (graphs, (start, end) CUDA
+        events) around the whole sequence; the caller synchronises."""
+        dev = self.device
+        if graphs is None:
+            graphs = []
+            for _ in range(2):
+                fd = torch.empty(host_features[0].shape, dtype=torch.bfloat16, device=dev)
+                fd.copy_(host_features[0])
+                out = torch.empty(host_outs[0].shape, dtype=torch.float32, device=dev)
+                g, _ = self.capture(fd, feature_lens, out=out)
+                graphs.append((g, fd, out))
+        comp = torch.cuda.current_stream(dev)
+        copy = torch.cuda.Stream(dev)
+        h2d = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        d2h = [torch.cuda.Event() for _ in range(2)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = len(host_features)
+        copy.wait_stream(comp)
+        start.record(copy)
+        with torch.cuda.stream(copy):
+            graphs[0][1].copy_(host_features[0], non_blocking=True)
+        h2d[0].record(copy)
+        for i in range(n):
+            j, jn = i % 2, (i + 1) % 2
+            if i + 1 < n:  # next batch in, once batch i - 1 no longer reads that buffer
+                if i >= 1:
+                    copy.wait_event(done[jn])
+                with torch.cuda.stream(copy):
+                    graphs[jn][1].copy_(host_features[i + 1], non_blocking=True)
+                h2d[jn].record(copy)
+            comp.wait_event(h2d[j])
+            if i >= 2:  # batch i - 2's result has left this output buffer
+                comp.wait_event(d2h[j])
+            if before_each is not None:
+                before_each()
+            graphs[j][0].replay()
+            done[j].record(comp)
+            copy.wait_event(done[j])
+            with torch.cuda.stream(copy):
+                host_outs[i].copy_(graphs[j][2], non_blocking=True)
+            d2h[j].record(copy)
+        end.record(copy)
+        comp.wait_stream(copy)
+        return graphs, (start, end)
+
     def check(self) -> int:
         """Device status of the latest call on this encoder's workspace."""
         return A.aut_check(self._ws.data_ptr()) if self._ws is not None else A.AUT_OK

@@ -285,24 +285,28 @@ def our_arm(args, rank, world, local_rank):
     gemm_avg_ms = gemm_ms / gemm_launches
     achieved = gemm_flops / gemm_launches / (gemm_avg_ms / 1e3) / 1e12
 
-    # End to end through the public API: pinned host features in, result back out.
+    # End to end through the public API: every step copies its features in from
+    # pinned host memory and its fp32 result back out; the copies of steps
+    # i - 1 and i + 1 overlap step i's compute (Encoder.encode_stream).
     h_feats = fd.cpu().pin_memory()
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-
-    def e2e_step():
-        fd.copy_(h_feats, non_blocking=True)
-        step()
-        h_out.copy_(out, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    e2e_ms = timed(e2e_step, args.steps)
-    e2e_total = sum(e2e_ms)
+    h_outs = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    graphs, _ = enc.encode_stream([h_feats] * 3, lens, [h_outs[i % 2] for i in range(3)],
+                                  before_each=flush.zero_)
+    torch.cuda.synchronize()
+    barrier()
+    _, (e0, e1) = enc.encode_stream([h_feats] * args.steps, lens,
+                                    [h_outs[i % 2] for i in range(args.steps)], graphs=graphs,
+                                    before_each=flush.zero_)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_total = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_total = float(t.item())
     e2e_value = world * audio_s * args.steps / (e2e_total / 1e3)
+    h_out = h_outs[0]
+    del graphs
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -346,7 +350,10 @@ def our_arm(args, rank, world, local_rank):
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": h_feats.numel() * h_feats.element_size(),
                     "d2h_bytes_per_step": h_out.numel() * h_out.element_size(),
-                    "ms_per_step": e2e_total / args.steps},
+                    "ms_per_step": e2e_total / args.steps,
+                    "copies": "each step's host-to-device and device-to-host copies run on a "
+                              "second stream, overlapping the neighbouring steps' compute; "
+                              "the L2 flush before every step is inside the timed region"},
             "gpu_launches": launches * args.steps,
             "device_status": A.status_string(status),
             "clocks": clocks,
