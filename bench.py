@@ -157,6 +157,25 @@ def oracle_sample(workload, lens, seconds_wanted=30.0):
     return out
 
 
+def layout_counts(cfg, lens):
+    """(total tokens, windows, chunks) of a batch, from the oracle's planner
+    (the reference arm runs none of the library)."""
+    import oracle as O
+    lay = O.plan(cfg, lens)
+    return lay.total_tokens, len(lay.cu_seqlens) - 1, len(lay.chunks)
+
+
+def workload_config(args, world, lens, T, nW, nch):
+    """The `config` object of the JSON line (both arms)."""
+    cfg = S.WORKLOADS[args.workload]
+    return {"workload": args.workload, "requests": len(lens), "frames": sum(lens),
+            "audio_seconds": sum(lens) / 100.0, "total_tokens": T, "windows": nW,
+            "chunks": nch, "d_model": cfg.d_model, "layers": cfg.encoder_layers,
+            "l2": "256 MiB buffer written between timed steps (outside the events)",
+            "launch": "CUDA graph of the whole forward" if args.graph else "eager",
+            "parallelism": f"dp{world} (weak: one batch per GPU)"}
+
+
 def reference_arm(args, rank, world):
     """The oracle as it stands, timed on the host cores; each step encodes one
     8 s window of the workload's first request."""
@@ -177,7 +196,8 @@ def reference_arm(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(ts) / len(ts),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": {"workload": args.workload},
+            "data": "synthetic",
+            "config": workload_config(args, world, lens_all, *layout_counts(cfg, lens_all)),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -327,12 +347,7 @@ def our_arm(args, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "requests": len(lens), "frames": sum(lens),
-                       "audio_seconds": audio_s, "total_tokens": T, "windows": nW,
-                       "chunks": nch, "d_model": cfg.d_model, "layers": cfg.encoder_layers,
-                       "l2": "256 MiB buffer written between timed steps (outside the events)",
-                       "launch": "CUDA graph of the whole forward" if args.graph else "eager",
-                       "parallelism": f"dp{world} (weak: one batch per GPU)"},
+            "config": workload_config(args, world, lens, T, nW, nch),
             "tokens_per_s": tokens_s,
             "tflops": flops / (ms / 1e3) / 1e12,
             "pct_bf16_peak": 100 * flops / (ms / 1e3) / 1e12 / pk,
