@@ -393,12 +393,20 @@ def sweep(args):
     pk = peaks()[0]
     rng = np.random.default_rng(S.SEED_LENGTHS + 7)
     pool = [int(round(100 * np.exp(rng.uniform(np.log(0.5), np.log(60.0))))) for _ in range(4096)]
-    for target in (1000, 2000, 5000, 10000, 20000, 50000, 100000, 200000):
+    for target in (1000, 2000, 4000, 8000, 16000, 32000, 64000, 100000, 128000, 200000):
+        # Requests from the pool until the next one would pass the target, then
+        # one request of exactly the missing k tokens: 100 floor(k / 13) +
+        # 8 (k mod 13) frames gives 13 floor(k / 13) + (k mod 13) tokens.
         lens, T = [], 0
-        while T < target:
+        while True:
+            t_next = enc.plan(lens + [pool[len(lens)]])[2]
+            if t_next > target:
+                break
             lens.append(pool[len(lens)])
-            if sum(lens) * 0.13 >= target or len(lens) % 32 == 0:
-                T = enc.plan(lens)[2]
+            T = t_next
+        k = target - T
+        if k > 0:
+            lens.append(100 * (k // 13) + 8 * (k % 13))
         feats = S.features(lens, seed=S.SEED_FEATURES)
         fd = enc.features_to_device(feats)
         _, cu, T, nW, nch = enc.plan(lens)
