@@ -121,10 +121,11 @@ GemmStatus dispatch(int bn, int cg, const CUtensorMap &ta, const CUtensorMap &tb
 bool pair_ok(int bn) { return bn == 64 || bn == 128 || bn == 192 || bn == 240 || bn == 256; }
 
 // Tile shape for a plain GEMM: the (width, CTAs per MMA) with the fewest waves
-// x per-tile time.  A tile keeps each of its SMs busy for ~128 x (BN + overhead)
-// MMA rows-columns; a CTA pair streams a third less operand data per FLOP,
-// which is what bounds single-SM tiles here (L2-to-SM bandwidth), so it is
-// credited as 4/6 of the single-SM time.
+// x per-tile time.  Per k-block a tile costs about (BN + 512) column-units:
+// the A tile arrives whatever the width, so halving BN saves far less than
+// half (measured on B200: a 256 x 128 pair k-block takes ~0.32 us against
+// ~0.37 us at 256 x 256).  A CTA pair streams a third less operand data per
+// FLOP than a single SM, so it is credited as 4/6 of the single-SM time.
 void choose_tile(int M, int N, int sms, bool allow_pair, int *bn_out, int *cg_out) {
     static const int cand[] = {256, 128, 64, 32, 16};
     long best_cost = -1;
@@ -138,7 +139,7 @@ void choose_tile(int M, int N, int sms, bool allow_pair, int *bn_out, int *cg_ou
             const long tiles = mt * (N / bn);
             const long slots = sms / cg;
             const long waves = (tiles + slots - 1) / slots;
-            const long cost = waves * 128 * (bn + 32) * (cg == 2 ? 4 : 6);
+            const long cost = waves * (bn + 512) * (cg == 2 ? 4 : 6);
             if (best_cost < 0 || cost < best_cost) {
                 best_cost = cost;
                 *bn_out = bn;
