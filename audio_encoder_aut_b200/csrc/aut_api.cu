@@ -120,9 +120,11 @@ struct Ctx {
 };
 
 aut_status linear(const Ctx &c, const void *a, const void *w, const void *b, void *out, int M,
-                  int N, int K, int epi, int kind, int ldo = 0, bool f16 = false) {
+                  int N, int K, int epi, int kind, int ldo = 0, bool f16 = false,
+                  int f16_col = 1 << 30) {
     LinearLaunch L{};
     L.f16 = f16;
+    L.f16_col = f16_col;
     L.a = a;
     L.w = w;
     L.bias = b;
@@ -241,9 +243,13 @@ aut_status run_encode(const Ctx &c, float *x, int T, int nW, int n_layers, void 
         const aut_layer_weights &lw = c.w->layers[l];
         AUT_TRY(cuda_status(launch_layernorm(x, lw.ln1_w, lw.ln1_b, xn, T, d, cfg->ln_eps, c.st)));
         AUT_TRY(c.mark(AUT_K_LAYERNORM));
-        AUT_TRY(linear(c, xn, lw.qkv_w, lw.qkv_b, qkv, T, 3 * d, d, kEpiBf16, AUT_K_QKV));
+        // With the tensor-core attention the qkv GEMM writes v as fp16, the
+        // type of the attention's P V product.
+        const bool v_f16 = window_attention_uses_tc(d, cfg->heads, T);
+        AUT_TRY(linear(c, xn, lw.qkv_w, lw.qkv_b, qkv, T, 3 * d, d, kEpiBf16, AUT_K_QKV, 0, false,
+                       v_f16 ? 2 * d : 1 << 30));
         AUT_TRY(cuda_status(launch_window_attention(qkv, attn, cu, nW, d, cfg->heads, c.st, T,
-                                                    c.status)));
+                                                    c.status, v_f16)));
         AUT_TRY(c.mark(AUT_K_ATTENTION));
         // fp16 attention output against the fp16 copy of o_w
         const void *o_w16 = static_cast<const uint8_t *>(c.w->o_w_f16) + (size_t)l * d * d * 2;

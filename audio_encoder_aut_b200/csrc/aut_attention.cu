@@ -25,7 +25,8 @@
 //              significant bits, 8x finer than bf16) in the swizzled K-major
 //              layout the MMA reads, over the Q and K tiles the first MMA no
 //              longer needs; V converted in place to fp16 (saturating: bf16
-//              values beyond fp16's range clamp to +-65504); then O / rowsum
+//              values beyond fp16's range clamp to +-65504) unless the qkv
+//              GEMM already wrote it as fp16 (v_f16); then O / rowsum
 //              written as fp16 [T, d] (11 significant bits for the o_proj GEMM,
 //              which runs on fp16 operands; rows past the window's end are not
 //              written)
@@ -119,7 +120,7 @@ __device__ __forceinline__ void window_of(const int *cu, int w, int *s0, int *le
 
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_qkv, __half *__restrict__ out, const int *__restrict__ cu,
-    int n_windows, int heads, int d, float scale_log2e, int *status) {
+    int n_windows, int heads, int d, float scale_log2e, int *status, int v_f16) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -378,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
             // V rows the MMA reads, to fp16 in place (same positions, so the
             // swizzled layout is kept).  Reading V directly needs the TMA
             // barrier's phase observed by this thread (it completed long ago).
-            fail = !mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs);
-            if (!fail) {
+            fail = !v_f16 && !mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs);
+            if (!fail && !v_f16) {
                 uint4 *vv = reinterpret_cast<uint4 *>(st + 2 * kTileBytes);
                 for (int i = ctid; i < n16 * 128; i += 32 * kComputeWarps) {
                     uint4 u = vv[i];
@@ -433,7 +434,8 @@ int sm_count_cached() {
 }  // namespace
 
 cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu_dev, int n_windows,
-                                       int d, int heads, int T, int *status, cudaStream_t st) {
+                                       int d, int heads, int T, int *status, cudaStream_t st,
+                                       bool v_f16) {
     if (n_windows <= 0) return cudaSuccess;
     if (d / heads != kHd || T <= 0) return cudaErrorInvalidValue;
     static bool attr_done[64] = {};
@@ -454,7 +456,8 @@ cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu
     const long tiles = (long)n_windows * heads;
     const int grid = (int)std::min<long>(tiles, (long)kCtasPerSm * sm_count_cached());
     return launch_pdl(window_attn_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, 1, tm,
-                      static_cast<__half *>(out), cu_dev, n_windows, heads, d, scale_log2e, status);
+                      static_cast<__half *>(out), cu_dev, n_windows, heads, d, scale_log2e, status,
+                      v_f16 ? 1 : 0);
 }
 
 }  // namespace aut

@@ -172,6 +172,7 @@ GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
         return GemmStatus::kTensorMap;
     GemmArgs args{};
     args.f16 = L.f16 ? 1 : 0;
+    args.f16_col = L.f16_col;
     args.M = L.M;
     args.N = L.N;
     args.num_m_tiles = (L.M + 128 * cg - 1) / (128 * cg);
@@ -226,6 +227,7 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     if (!make_map(&ta, 4, L.planes, da, sa, ba) || !make_map(&tb, 3, L.w_tap, db, sb, bb))
         return GemmStatus::kTensorMap;
     GemmArgs args{};
+    args.f16_col = 1 << 30;
     args.M = (int)rows_total;
     args.N = L.C;
     const long slot_rows = (long)L.rows_per_tile * cg;

@@ -64,6 +64,9 @@ struct GemmArgs {
     // outputs (kEpiBf16, kEpiBf16Gelu, kEpiResidF32, kEpiF32) whose per-warp
     // column range is a whole number of 128-byte pieces.
     int tma_out;
+    // bf16 epilogues: output columns from here on are written as fp16 instead
+    // (the V part of qkv for the tensor-core attention); a multiple of 64.
+    int f16_col;
 };
 
 // BN: tile width of one MMA (N).  CG: CTAs per MMA (1, or 2 for a CTA pair
@@ -117,6 +120,21 @@ AUT_DEV void store_bf16x16(__nv_bfloat16 *p, const float (&v)[16]) {
     b.y = pack_bf16x2(v[10], v[11]);
     b.z = pack_bf16x2(v[12], v[13]);
     b.w = pack_bf16x2(v[14], v[15]);
+    reinterpret_cast<uint4 *>(p)[0] = a;
+    reinterpret_cast<uint4 *>(p)[1] = b;
+}
+
+// The same as fp16 (saturating at +-65504).
+AUT_DEV void store_f16x16(__nv_bfloat16 *p, const float (&v)[16]) {
+    uint4 a, b;
+    a.x = pack_f16x2_sat(v[0], v[1]);
+    a.y = pack_f16x2_sat(v[2], v[3]);
+    a.z = pack_f16x2_sat(v[4], v[5]);
+    a.w = pack_f16x2_sat(v[6], v[7]);
+    b.x = pack_f16x2_sat(v[8], v[9]);
+    b.y = pack_f16x2_sat(v[10], v[11]);
+    b.z = pack_f16x2_sat(v[12], v[13]);
+    b.w = pack_f16x2_sat(v[14], v[15]);
     reinterpret_cast<uint4 *>(p)[0] = a;
     reinterpret_cast<uint4 *>(p)[1] = b;
 }
@@ -569,6 +587,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j >> 4][j & 15]);
                 } else {
+                    const bool as_f16 = n_first + p * pcols >= args.f16_col;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {  // 32 columns at a time
                         float v[2][16];
@@ -588,7 +607,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             }
 #pragma unroll
                             for (int j = 0; j < 8; ++j)
-                                w[16 * h + 8 * i + j] = pack_bf16x2(v[i][2 * j], v[i][2 * j + 1]);
+                                w[16 * h + 8 * i + j] =
+                                    as_f16 ? pack_f16x2_sat(v[i][2 * j], v[i][2 * j + 1])
+                                           : pack_bf16x2(v[i][2 * j], v[i][2 * j + 1]);
                         }
                     }
                 }
@@ -656,7 +677,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (!resid) add_bias16(v, args.bias, n0);
                     switch (args.epi) {
                         case kEpiBf16:
-                            store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
+                            if (n0 >= args.f16_col)
+                                store_f16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
+                            else
+                                store_bf16x16(reinterpret_cast<__nv_bfloat16 *>(args.out) + dst_row + n0, v);
                             break;
                         case kEpiBf16Gelu:
                         case kEpiConvPlanes:

@@ -65,12 +65,17 @@ cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void 
                              float eps, cudaStream_t st, bool split = false);
 cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st);
 cudaError_t launch_to_f16(const void *src, void *dst, size_t n, cudaStream_t st);
+// v_f16: the v third of qkv already holds fp16 (the qkv GEMM wrote it so); only
+// the head_dim-64 tensor-core path (T > 0) accepts it.
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                     int d, int heads, cudaStream_t st, int T = -1,
-                                    int *status = nullptr);
+                                    int *status = nullptr, bool v_f16 = false);
+// Whether launch_window_attention takes the tensor-core path.
+inline bool window_attention_uses_tc(int d, int heads, int T) { return d / heads == 64 && T > 0; }
 // tcgen05 variant for head_dim 64 (aut_attention.cu); T = rows of qkv.
 cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu_dev, int n_windows,
-                                       int d, int heads, int T, int *status, cudaStream_t st);
+                                       int d, int heads, int T, int *status, cudaStream_t st,
+                                       bool v_f16 = false);
 // bf16 tensor map with 128-byte swizzle (aut_gemm.cu): dims innermost first,
 // strides in bytes for dims 1.., box in elements.
 bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
@@ -99,6 +104,7 @@ struct LinearLaunch {
     int fault_inject;
     bool single_cta = false;  // force one CTA per MMA (no CTA pairs)
     bool f16 = false;         // A and W are fp16 instead of bf16
+    int f16_col = 1 << 30;    // kEpiBf16: output columns from here on written as fp16
 };
 GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st);
 
