@@ -122,9 +122,10 @@ size_t aut_prepared_bytes(const aut_config *cfg);
  * Writes into `dst` (device, dst_bytes >= aut_prepared_bytes) the tap-major conv2
  * and conv3 weights, conv_out's columns reordered to the stem's output order,
  * the sinusoid table (aut_encoder page, module docstring: the same 13 positions
- * for every chunk) and the K-repeated o_proj and projector weights.  Copies
- * `src` into `*prepared` and points the seven prepared fields into `dst`.  Asynchronous on `stream`; src stays owned by the caller and
- * must stay alive while `prepared` is used. */
+ * for every chunk), every layer's o_proj weight converted to fp16, and the
+ * K-repeated projector weights.  Copies `src` into `*prepared` and points the
+ * seven prepared fields into `dst`.  Asynchronous on `stream`; src stays owned
+ * by the caller and must stay alive while `prepared` is used. */
 aut_status aut_prepare_weights(const aut_config *cfg, const aut_weights *src, void *dst,
                                size_t dst_bytes, aut_weights *prepared, aut_stream_t stream);
 
