@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (args.tma_out) tma_prefetch_desc(&tmC);
     }
     if (warp == 1) {
         if constexpr (CG == 2) {
@@ -749,7 +750,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         if (!ok && lane == 0) gemm_signal_abort(args, abort_v);
-        if (args.tma_out && lane == 0) bulk_wait_all();  // stores complete before exit
+        // The staged stores have read shared memory before the block may exit;
+        // their global writes complete with the grid, before any dependent
+        // launch passes its griddepcontrol.wait.
+        if (args.tma_out && lane == 0) bulk_wait_read_all();
         if (x_pending) mbar_wait(my_xbar, xph, nullptr, lim);  // a residual load in flight lands
         __syncwarp();
     }
