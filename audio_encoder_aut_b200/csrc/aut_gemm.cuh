@@ -482,6 +482,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         };
         // Residual mode: accumulator `acc` <- x + bias over this thread's row and chunks.
         auto preload = [&](int tile, int acc, bool rel) {
+            __syncwarp();  // TMEM stores are warp-wide
             bool valid;
             size_t dst_row;
             int pos_row;
@@ -559,6 +560,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             for (int j = 0; j < 16; ++j) v[i][j] += r[i][j];
                     } else {
                         if (resid_drain && slab && p > 0 && lane == 0) load_x(tile, p * pcols);
+                        __syncwarp();  // the warp-wide TMEM wait needs every lane here
                         tc_wait_ld();
                         if (!resid || resid_drain) {
                             add_bias16(v[0], args.bias, n_first + p * pcols);
@@ -628,6 +630,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tma_store_2d(&tmC, stg, n_first + p * pcols, m0);
                     bulk_commit();
                 }
+                __syncwarp();  // converged again before the next warp-wide TMEM load
             }
         };
 
@@ -650,6 +653,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ok = false;
                 break;
             }
+            __syncwarp();  // lanes leave the wait loop separately; TMEM loads are warp-wide
             tc_fence_after();
             const int n_blk = tile % args.num_n_tiles;
             bool valid;
@@ -665,6 +669,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int c1 = c0 + 2;
                 const bool two = c1 < NC;  // warp-uniform
                 float v0[16], v1[16];
+                __syncwarp();  // lanes past the tile's valid rows skip ahead below
                 tmem_ld16(t_addr + c0 * 16, v0);
                 if (two) tmem_ld16(t_addr + c1 * 16, v1);
                 tc_wait_ld();
