@@ -77,3 +77,47 @@ def test_two_rank_sharded_forward_equals_unsharded(tmp_path):
     assert same_rows == 1.0
     # fp64; BLAS blocks shorter matrices differently, so rows agree to rounding
     assert err < 1e-12
+
+
+def test_shard_planner_properties_random():
+    """Random batches, window sizes, cut lengths and rank counts: the pieces
+    tile every request on window boundaries, their token counts add up to the
+    oracle's, every piece lands on exactly one rank, the LPT loads stay within
+    one piece of each other, and reassembling per-rank rows that carry their
+    own coordinates gives the unsharded packed order."""
+    rng = np.random.default_rng(123)
+    for trial in range(200):
+        nwi = 100 * int(rng.integers(1, 9))
+        lens = [int(x) for x in rng.integers(0, 6000, size=int(rng.integers(1, 12)))]
+        max_frames = int(rng.integers(nwi, 5000)) if trial % 3 else None
+        world = int(rng.integers(1, 6))
+        ps = SH.pieces(lens, nwi, max_frames=max_frames)
+        for r, n in enumerate(lens):
+            mine = sorted((p.frame0, p.frames) for p in ps if p.request == r)
+            covered = 0
+            for f0, nf in mine:
+                assert f0 == covered and f0 % nwi == 0 and nf > 0
+                covered += nf
+            assert covered == n
+            assert sum(SH._tokens(p.frames) for p in ps if p.request == r) == \
+                O.tokens_for_frames(S.TINY, n)
+        shards = SH.assign(ps, world)
+        assert len(shards) == world
+        assert sorted(p for s in shards for p in s) == sorted(ps)
+        if ps:
+            loads = [sum(SH._tokens(p.frames) for p in s) for s in shards]
+            assert max(loads) - min(loads) <= max(SH._tokens(p.frames) for p in ps)
+        # each rank's "output" rows hold (request, token index within the request)
+        outputs = []
+        for s in shards:
+            rows = []
+            for p in s:
+                t0 = SH._tokens(p.frame0)
+                rows += [(p.request, t0 + i) for i in range(SH._tokens(p.frames))]
+            outputs.append(np.array(rows, dtype=np.int64).reshape(-1, 2))
+        got = SH.reassemble(lens, shards, outputs)
+        want = [(r, i) for r, n in enumerate(lens) for i in range(O.tokens_for_frames(S.TINY, n))]
+        if want:
+            assert got.tolist() == [list(w) for w in want]
+        else:
+            assert got is None
