@@ -88,6 +88,12 @@ _SIGNATURES = {
                                        POINTER(c_int32), c_int32, c_void_p, c_size_t, c_void_p]),
     "aut_window_attention_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                                POINTER(c_int32), c_int32, c_void_p]),
+    "aut_logmel": (c_int32, [c_void_p, ctypes.c_int64, POINTER(c_int32), c_int32, c_void_p,
+                             c_int32, POINTER(c_int32), c_void_p, c_size_t, c_void_p]),
+    "aut_logmel_workspace_bytes": (c_size_t, [c_int32, c_int32]),
+    "aut_inject_audio": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_int32,
+                                   c_int32, c_void_p, c_size_t, c_void_p]),
+    "aut_inject_workspace_bytes": (c_size_t, [c_int32]),
     "aut_check": (c_int32, [c_void_p]),
     "aut_check_status_word": (c_int32, [c_void_p]),
     "aut_status_string": (c_char_p, [c_int32]),
@@ -231,6 +237,29 @@ def aut_window_attention_noalloc(qkv: int, out: int, T: int, d: int, heads: int,
     device array; see include/aut.h for its limits)."""
     return lib().aut_window_attention_noalloc(qkv, out, T, d, heads, _i32(cu_seqlens),
                                               len(cu_seqlens) - 1, stream)
+
+
+def aut_logmel(waveform: int, s_max: int, sample_lens, features: int, t_max: int,
+               workspace: int, ws_bytes: int, stream: int):
+    """-> (status, feature_lens)."""
+    fl = (c_int32 * max(1, len(sample_lens)))()
+    st = lib().aut_logmel(waveform, s_max, _i32(sample_lens), len(sample_lens), features, t_max,
+                          fl, workspace, ws_bytes, stream)
+    return st, list(fl)[:len(sample_lens)]
+
+
+def aut_logmel_workspace_bytes(n_req: int, t_max: int) -> int:
+    return lib().aut_logmel_workspace_bytes(n_req, t_max)
+
+
+def aut_inject_audio(embeds: int, token_ids: int, L: int, audio_pad_id: int, audio: int, T: int,
+                     D: int, workspace: int, ws_bytes: int, stream: int) -> int:
+    return lib().aut_inject_audio(embeds, token_ids, L, audio_pad_id, audio, T, D, workspace,
+                                  ws_bytes, stream)
+
+
+def aut_inject_workspace_bytes(L: int) -> int:
+    return lib().aut_inject_workspace_bytes(L)
 
 
 def aut_check(workspace: int) -> int:

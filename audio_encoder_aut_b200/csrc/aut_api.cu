@@ -10,7 +10,7 @@
 //   per layer: LN1 -> qkv (GEMM + bias) -> window attention -> o_proj (GEMM +
 //     bias + residual) -> LN2 -> fc1 (GEMM + bias + GELU) -> fc2 (GEMM + bias +
 //     residual)
-//   final LN -> proj1 (GEMM + bias + GELU) -> proj2 (GEMM + bias) -> out (bf16)
+//   final LN -> proj1 (GEMM + bias + GELU) -> proj2 (GEMM + bias) -> out (fp32)
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -507,17 +507,21 @@ extern "C" aut_status aut_window_attention(const void *qkv, void *out, int32_t T
     if (T > 0 && (!qkv || !out)) return AUT_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15u)
         return AUT_ERR_INVALID_ARG;
-    if (!workspace || ws_bytes < (size_t)(num_windows + 1) * 4) return AUT_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < (size_t)(num_windows + 2) * 4) return AUT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 3u) return AUT_ERR_INVALID_ARG;
     if (T == 0) return AUT_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    AUT_TRY(cuda_status(launch_upload(cu_seqlens, (size_t)num_windows + 1,
-                                      static_cast<int32_t *>(workspace), st)));
-    return cuda_status(launch_window_attention(qkv, out, static_cast<const int *>(workspace),
-                                               num_windows, d, heads, st, T));
+    // Workspace words: [0] the status word (cleared here), [1 ..] cu_seqlens.
+    std::vector<int32_t> words(1, 0);
+    words.insert(words.end(), cu_seqlens, cu_seqlens + num_windows + 1);
+    int32_t *ws = static_cast<int32_t *>(workspace);
+    AUT_TRY(cuda_status(launch_upload(words.data(), words.size(), ws, st)));
+    return cuda_status(
+        launch_window_attention(qkv, out, ws + 1, num_windows, d, heads, st, T, ws));
 }
 
 extern "C" aut_status aut_check_status_word(int32_t *status) {
-    if (!status) return AUT_ERR_INVALID_ARG;
+    if (!status) AUT_TRY(noalloc_status_word(&status));
     int32_t v = 0;
     if (cudaMemcpy(&v, status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return AUT_ERR_CUDA;
     const int32_t zero = 0;

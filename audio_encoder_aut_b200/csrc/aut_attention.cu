@@ -419,18 +419,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
     }
 }
 
-int sm_count_cached() {
-    static int n[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!n[dev]) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        n[dev] = v > 0 ? v : 1;
-    }
-    return n[dev];
-}
-
 }  // namespace
 
 cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu_dev, int n_windows,
@@ -438,15 +426,8 @@ cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu
                                        bool v_f16) {
     if (n_windows <= 0) return cudaSuccess;
     if (d / heads != kHd || T <= 0) return cudaErrorInvalidValue;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(
-            window_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+    const cudaError_t e = smem_attr_once<window_attn_tc_kernel>(kSmem);
+    if (e != cudaSuccess) return e;
     CUtensorMap tm;
     const uint64_t dims[2] = {(uint64_t)3 * d, (uint64_t)T};
     const uint64_t strides[1] = {(uint64_t)3 * d * 2};

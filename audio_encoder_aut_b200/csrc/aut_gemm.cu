@@ -61,12 +61,7 @@ bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const
 
 namespace {
 
-int sm_count() {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 1;
-}
+int sm_count() { return sm_count_cached(); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -75,17 +70,8 @@ GemmStatus run(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &
                const GemmArgs &args,
                cudaStream_t st) {
     using Cfg = GemmCfg<BN, CG>;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) return GemmStatus::kLaunch;
-    if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<BN, CG>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg::SMEM_BYTES) != cudaSuccess)
-            return GemmStatus::kLaunch;
-        attr_done[dev] = true;
-    }
+    if (smem_attr_once<gemm_tc_kernel<BN, CG>>(Cfg::SMEM_BYTES) != cudaSuccess)
+        return GemmStatus::kLaunch;
     const int tiles = args.num_m_tiles * args.num_n_tiles;
     const int groups = std::min(tiles, sm_count() / CG);
     const cudaError_t e = launch_pdl(gemm_tc_kernel<BN, CG>, dim3(groups * CG), dim3(kGemmThreads),
@@ -158,7 +144,7 @@ GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
     if (!aligned16(L.a) || !aligned16(L.w) || !aligned16(L.out) || (L.bias && !aligned16(L.bias)))
         return GemmStatus::kBadShape;
     int bn = 0, cg = 1;
-    choose_tile(L.M, L.N, sm_count(), L.fault_inject == 0 && !L.single_cta, &bn, &cg);
+    choose_tile(L.M, L.N, sm_count(), !L.single_cta, &bn, &cg);
     if (!bn) return GemmStatus::kBadShape;
     CUtensorMap ta, tb;
     const cuuint64_t da[2] = {(cuuint64_t)L.K, (cuuint64_t)L.M};

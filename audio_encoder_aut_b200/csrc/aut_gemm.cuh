@@ -90,7 +90,7 @@ struct GemmCfg {
     // a whole number of 32-column fp32 pieces (no other width can use it, and
     // shared memory left unallocated serves as L1 cache).
     static constexpr int STAGING_BYTES = (BN / 2) % 32 == 0 ? 8 * 4096 : 0;
-    static constexpr int BAR_BYTES = 256;
+    static constexpr int BAR_BYTES = 384;
     static constexpr int SMEM_BYTES =
         1024 /*alignment slack*/ + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
@@ -174,7 +174,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *tempty = tfull + 2;
     uint64_t *mma_done = tempty + 2;
     uint64_t *xbar = mma_done + 1;  // [8] per epilogue warp: residual piece landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xbar + kEpilogueWarps);
+    // [STAGES] odd CTA of a pair: the even CTA has armed the stage's `full`
+    // barrier for the phase the odd CTA is about to load into.
+    uint64_t *armed = xbar + kEpilogueWarps;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(armed + STAGES);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     pdl_trigger();
@@ -192,6 +195,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(mma_done, 1);
         for (int w = 0; w < kEpilogueWarps; ++w) mbar_init(xbar + w, 1);
+        for (int st = 0; st < STAGES; ++st) mbar_init(armed + st, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -226,11 +230,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // ------------------------------------------------ TMA producer --
             // Both CTAs of a pair load their own A rows and B half; the loads of
             // both complete on the even CTA's `full` barrier, which the even CTA
-            // arms with the pair's byte count.
+            // arms with the pair's byte count and then reports armed to the odd
+            // CTA.  The odd CTA loads into a phase only once it is armed, so
+            // every copy either CTA has in flight is counted on a phase the even
+            // CTA waits for before the pair may exit.
             const uint32_t a_bytes =
                 args.conv ? 128u * args.conv_rows * args.conv_cols : (uint32_t)Cfg::A_BYTES;
             auto arm = [&](int stage) {
-                if (rank == 0) mbar_arrive_expect_tx(full + stage, CG * (a_bytes + Cfg::B_BYTES));
+                if (rank == 0) {
+                    mbar_arrive_expect_tx(full + stage, CG * (a_bytes + Cfg::B_BYTES));
+                    if constexpr (CG == 2) mbar_arrive_cluster(map_to_rank(armed + stage, 1));
+                }
             };
             // Weights (B): k-block kb of the tile whose B rows start at b_row.
             auto load_b = [&](int stage, int kb, int b_row) {
@@ -289,6 +299,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (rank == 1 && !mbar_wait(armed + stage, phase, abort_v, lim)) {
+                        ok = false;
+                        break;
+                    }
                     if (skip) {
                         skip = false;  // injected fault: this stage is never filled
                     } else {
@@ -306,14 +320,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             if (!ok) gemm_signal_abort(args, abort_v);
             if (rank == 0) {
-                // The last load issued on every stage has landed before the block may exit.
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued >> s & 1u) mbar_wait(full + s, parity >> s & 1u, nullptr, lim);
-            } else if (!ok) {
-                // The odd CTA's loads complete on the even CTA's barriers; after a
-                // failure give its copies in flight time to land before exiting.
+                // The last load issued on every stage (the odd CTA's included) has
+                // landed before the pair may exit: the odd CTA leaves only through
+                // the cluster barrier at the end, which this CTA reaches after
+                // these waits.  After a failure a phase whose odd half was never
+                // issued does not complete; one shared time limit bounds them all.
                 const uint64_t t0 = global_timer_ns();
-                while (global_timer_ns() - t0 < 200000ull) {
+                for (int s = 0; s < STAGES; ++s) {
+                    const uint64_t used = global_timer_ns() - t0;
+                    if ((issued >> s & 1u) && used < lim)
+                        mbar_wait(full + s, parity >> s & 1u, nullptr, lim - used);
                 }
             }
         }
@@ -562,12 +578,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (resid_drain && slab && p > 0 && lane == 0) load_x(tile, p * pcols);
                         __syncwarp();  // the warp-wide TMEM wait needs every lane here
                         tc_wait_ld();
-                        if (!resid || resid_drain) {
+                        if (!resid) {
                             add_bias16(v[0], args.bias, n_first + p * pcols);
                             add_bias16(v[1], args.bias, n_first + p * pcols + 16);
                         }
-                        if (resid_drain && slab) {  // + the residual piece from the box
-                            if (!mbar_wait(my_xbar, xph, abort_v, lim)) {
+                        if (resid_drain && slab) {
+                            // + (residual piece from the box + bias): the same order
+                            // of additions as the single-tile path, acc + (x + b),
+                            // so that a row's result does not depend on how many
+                            // tiles its launch has.
+                            if (!mbar_wait_warp(my_xbar, xph, abort_v, lim)) {
                                 ok = false;
                                 gemm_signal_abort(args, abort_v);
                             } else {
@@ -575,16 +595,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             }
                             xph ^= 1u;
                             const uint8_t *row = stg + lane * 128;
+                            float xr[2][16];
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
                                 const float4 x4 = *reinterpret_cast<const float4 *>(
                                     row + ((j ^ (lane & 7)) << 4));
-                                float *q = &v[j >> 2][(j & 3) * 4];
-                                q[0] += x4.x;
-                                q[1] += x4.y;
-                                q[2] += x4.z;
-                                q[3] += x4.w;
+                                float *q = &xr[j >> 2][(j & 3) * 4];
+                                q[0] = x4.x;
+                                q[1] = x4.y;
+                                q[2] = x4.z;
+                                q[3] = x4.w;
                             }
+                            add_bias16(xr[0], args.bias, n_first + p * pcols);
+                            add_bias16(xr[1], args.bias, n_first + p * pcols + 16);
+#pragma unroll
+                            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) v[i][j] += xr[i][j];
                         }
                     }
 #pragma unroll
@@ -649,11 +676,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (resid_drain && lane == 0 &&  // first residual piece lands during the mainloop
                 ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32 < args.M)
                 load_x(tile, 0);
-            if (!mbar_wait(tfull + acc, acc_phase, abort_v, lim)) {
+            __syncwarp();  // lane 0's residual load above is the only divergent step
+            if (!mbar_wait_warp(tfull + acc, acc_phase, abort_v, lim)) {
                 ok = false;
                 break;
             }
-            __syncwarp();  // lanes leave the wait loop separately; TMEM loads are warp-wide
             tc_fence_after();
             const int n_blk = tile % args.num_n_tiles;
             bool valid;

@@ -52,4 +52,8 @@ struct WorkspaceLayout {
 };
 WorkspaceLayout workspace_layout(const aut_config *c, int64_t T, int64_t nW, int64_t n_ch);
 
+// Device address, on the current device, of the status word the
+// allocation-free window attention writes (aut_noalloc.cu).
+aut_status noalloc_status_word(int32_t **out);
+
 }  // namespace aut

@@ -454,6 +454,20 @@ __global__ void upload_words_kernel(const UploadPayload p, int32_t *dst) {
 }
 
 // ------------------------------------------------------------ launchers ----
+int sm_count_cached() {
+    static std::mutex mu;
+    static int n[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!n[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 1;
+    }
+    return n[dev];
+}
+
 cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int chunk_base,
                          int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
                          int C, cudaStream_t st) {
@@ -508,15 +522,8 @@ template <int HD>
 cudaError_t run_window_attention(const bf16 *q, __half *o, const int *cu_dev, int n_windows, int d,
                                  int heads, float scale_log2e, cudaStream_t st) {
     constexpr int smem = 2 * kMaxWindowTokens * (HD + 8) * (int)sizeof(bf16);
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(window_attn_kernel<HD>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+    const cudaError_t e = smem_attr_once<window_attn_kernel<HD>>(smem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(window_attn_kernel<HD>, dim3(n_windows, heads), dim3(32 * kAttnWarps), smem, st,
                       1, q, o, cu_dev, d, scale_log2e);
 }

@@ -7,9 +7,32 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <utility>
 
 namespace aut {
+
+// Raises `Kernel`'s dynamic shared-memory limit to `bytes`, once per device;
+// safe when several host threads make their first call at the same time.
+template <auto Kernel>
+cudaError_t smem_attr_once(int bytes) {
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        done[dev] = true;
+    }
+    return cudaSuccess;
+}
+
+// Multiprocessor count of the current device (cached per device, thread-safe).
+int sm_count_cached();
 
 // Launches a forward-path kernel that may start while the previous kernel in
 // the stream finishes (programmatic dependent launch); the kernel itself waits

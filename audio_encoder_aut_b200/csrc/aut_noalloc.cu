@@ -19,12 +19,14 @@
 namespace aut {
 namespace {
 
-constexpr int kNoAllocMaxWindows = 32767;  // cu_seqlens of at most 32768 entries (128 KiB)
+constexpr int kNoAllocMaxWindows = 32766;  // status word + cu_seqlens: 32768 words (128 KiB)
 
+// Word 0 is the call's status word (a bounded wait that runs out writes
+// AUT_ERR_TIMEOUT there), words 1 .. num_windows + 1 the uploaded cu_seqlens.
 // Every GPU that loads the library holds this array until the process exits.
 // All calls share it: calls that overlap on the GPU (different streams without
 // ordering between them) race on it.
-__device__ __align__(256) int32_t g_cu_seqlens_scratch[kNoAllocMaxWindows + 1];
+__device__ __align__(256) int32_t g_cu_seqlens_scratch[kNoAllocMaxWindows + 2];
 
 // The array's device address for the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
@@ -46,6 +48,9 @@ aut_status scratch_for_current_device(int32_t **out) {
 }
 
 }  // namespace
+
+aut_status noalloc_status_word(int32_t **out) { return scratch_for_current_device(out); }
+
 }  // namespace aut
 
 extern "C" aut_status aut_window_attention_noalloc(const void *qkv, void *out, int32_t T, int32_t d,
@@ -70,11 +75,14 @@ extern "C" aut_status aut_window_attention_noalloc(const void *qkv, void *out, i
     if (st != AUT_OK) return st;
     if (T == 0) return AUT_OK;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // The whole array prefix the kernel reads is rewritten on every call; nothing
-    // needs to start at zero.
-    if (launch_upload(cu_seqlens, (size_t)num_windows + 1, scratch, s) != cudaSuccess)
-        return AUT_ERR_CUDA;
-    return launch_window_attention(qkv, out, scratch, num_windows, d, heads, s, T) == cudaSuccess
+    // One upload rewrites, in stream order, everything the kernel reads: the
+    // status word (cleared to 0) and the whole cu_seqlens prefix.  Entries past
+    // it, left by an earlier call with more windows, are never read.
+    std::vector<int32_t> words(1, 0);
+    words.insert(words.end(), cu_seqlens, cu_seqlens + num_windows + 1);
+    if (launch_upload(words.data(), words.size(), scratch, s) != cudaSuccess) return AUT_ERR_CUDA;
+    return launch_window_attention(qkv, out, scratch + 1, num_windows, d, heads, s, T, scratch) ==
+                   cudaSuccess
                ? AUT_OK
                : AUT_ERR_CUDA;
 }

@@ -68,6 +68,15 @@ AUT_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint
     }
 }
 
+// mbar_wait for a whole converged warp, with one answer for every lane: each
+// lane polls on its own, so near a time-out or an abort some lanes could see
+// the phase complete and others give up; the vote makes the warp leave (or
+// carry on) together, as the warp-wide tcgen05 operations after it require.
+AUT_DEV bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort, uint64_t limit_ns) {
+    const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // -------------------------------------------------------------------- TMA --
 AUT_DEV void tma_prefetch_desc(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -68,6 +68,7 @@ class Encoder:
             self.prepared = A.aut_prepare_weights(self.c, self._src, self._prepared_buf.data_ptr(),
                                                   nbytes, current_stream_handle(dev))
         self._ws = None
+        self._lm_ws = None
 
     # ------------------------------------------------------------------
     def plan(self, feature_lens):
@@ -80,6 +81,23 @@ class Encoder:
         if self._ws is None or self._ws.numel() < need:
             self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
         return self._ws
+
+    def logmel(self, waveform: torch.Tensor, sample_lens, t_max: int | None = None):
+        """16 kHz mono waveform, device fp32 [B, S_max] -> (features bf16
+        [B, 128, T_max] on the device, feature_lens), through aut_logmel."""
+        waveform = waveform.contiguous()
+        frames = [int(n) // 160 for n in sample_lens]
+        t = max(frames + [1]) if t_max is None else t_max
+        feats = torch.empty((len(sample_lens), 128, t), dtype=torch.bfloat16, device=self.device)
+        need = A.aut_logmel_workspace_bytes(len(sample_lens), t)
+        if self._lm_ws is None or self._lm_ws.numel() < need:
+            self._lm_ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        st, lens = A.aut_logmel(waveform.data_ptr(), waveform.shape[-1], sample_lens,
+                                feats.data_ptr(), t, self._lm_ws.data_ptr(), self._lm_ws.numel(),
+                                current_stream_handle(self.device))
+        if st != A.AUT_OK:
+            raise A.AutError(st, "aut_logmel")
+        return feats, lens
 
     def features_to_device(self, feats: np.ndarray) -> torch.Tensor:
         return _dev_bf16(feats, self.device)

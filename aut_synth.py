@@ -16,7 +16,7 @@ Conventions (PyTorch layouts, every parameter bf16-representable):
 
 Values are drawn in fp32 from numpy's PCG64 and rounded once to bf16
 (round-to-nearest-even); both the oracle and the GPU see the same rounded values.
-Seeds: lengths 0, features 1, weights 2.
+Seeds: lengths 0, features 1, weights 2, waveforms 3.
 """
 from __future__ import annotations
 
@@ -26,6 +26,7 @@ import numpy as np
 SEED_LENGTHS = 0
 SEED_FEATURES = 1
 SEED_WEIGHTS = 2
+SEED_WAVES = 3
 
 
 @dataclasses.dataclass(frozen=True)
@@ -192,3 +193,38 @@ def randomize_layernorm(w: dict, seed: int = 7) -> dict:
     d = w["ln_post_w"].shape[0]
     w["ln_post_w"], w["ln_post_b"] = g(d), b(d)
     return w
+
+
+def waveforms(n_samples: list[int], seed: int = SEED_WAVES, sample_rate: int = 16000) -> list:
+    """Speech-like 16 kHz mono stand-ins, one float64 array per request: a
+    voiced source (20 harmonics of a pitch that wanders over 90 - 250 Hz)
+    shaped by two random formant bumps that move every 0.25 s, a 3 - 6 Hz
+    syllable envelope with occasional pauses, and a little white noise
+    (peak amplitude about 0.3).  For front-end workloads only: the encoder's
+    own workloads start from features()."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for n in n_samples:
+        if n <= 0:
+            out.append(np.zeros(0))
+            continue
+        t = np.arange(n) / sample_rate
+        seg = max(1, int(0.25 * sample_rate))
+        n_seg = -(-n // seg) + 1
+        knots = np.arange(n_seg) * seg
+        f0 = np.interp(np.arange(n), knots, rng.uniform(90.0, 250.0, n_seg))
+        f1 = np.interp(np.arange(n), knots, rng.uniform(300.0, 900.0, n_seg))
+        f2 = np.interp(np.arange(n), knots, rng.uniform(900.0, 2500.0, n_seg))
+        phase = 2 * np.pi * np.cumsum(f0) / sample_rate
+        x = np.zeros(n)
+        for h in range(1, 21):
+            fh = h * f0
+            amp = (np.exp(-((fh - f1) / 150.0) ** 2) + 0.6 * np.exp(-((fh - f2) / 250.0) ** 2)
+                   + 0.05) / h
+            x += amp * np.sin(h * phase)
+        env = 0.5 + 0.5 * np.sin(2 * np.pi * rng.uniform(3.0, 6.0) * t + rng.uniform(0, 2 * np.pi))
+        gate = np.interp(np.arange(n), knots, (rng.uniform(size=n_seg) > 0.15).astype(float))
+        x = x * env * gate
+        x = 0.3 * x / max(1e-9, np.abs(x).max()) + 0.003 * rng.standard_normal(n)
+        out.append(x)
+    return out

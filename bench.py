@@ -11,9 +11,12 @@ input resident in HBM.  Prints one JSON line (rank 0).
 Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on
 the launching stream, with a 256 MiB buffer written between steps (L2 flush,
 outside the events); barrier + synchronize around the timed region; the
-device time is the max over ranks.  Weak scaling: every rank encodes its own
-batch of the same shape (different features, same weights); no collective is
-on the data path.
+device time is the max over ranks.  Weak scaling: with N ranks the job is N
+copies of the workload's requests, cut at window boundaries and assigned to
+the ranks by tokens (audio_encoder_aut_b200.shard); each rank encodes its
+shard, weights replicated; no collective is on the data path (only the timing
+maximum is reduced).  `--gpus N` outside a launcher starts the N processes
+itself.
 """
 from __future__ import annotations
 
@@ -165,15 +168,22 @@ def layout_counts(cfg, lens):
     return lay.total_tokens, len(lay.cu_seqlens) - 1, len(lay.chunks)
 
 
-def workload_config(args, world, lens, T, nW, nch):
+def workload_config(args, world, lens, T, nW, nch, impl="ours"):
     """The `config` object of the JSON line (both arms)."""
     cfg = S.WORKLOADS[args.workload]
-    return {"workload": args.workload, "requests": len(lens), "frames": sum(lens),
-            "audio_seconds": sum(lens) / 100.0, "total_tokens": T, "windows": nW,
-            "chunks": nch, "d_model": cfg.d_model, "layers": cfg.encoder_layers,
-            "l2": "256 MiB buffer written between timed steps (outside the events)",
-            "launch": "CUDA graph of the whole forward" if args.graph else "eager",
-            "parallelism": f"dp{world} (weak: one batch per GPU)"}
+    c = {"workload": args.workload, "requests": len(lens), "frames": sum(lens),
+         "audio_seconds": sum(lens) / 100.0, "total_tokens": T, "windows": nW,
+         "chunks": nch, "d_model": cfg.d_model, "layers": cfg.encoder_layers}
+    if impl == "reference":
+        c.update(launch="numpy oracle on the host cores (no GPU)", l2="not applicable (CPU)",
+                 parallelism="one process (rank 0)")
+    else:
+        c.update(l2="256 MiB buffer written between timed steps (outside the events)",
+                 launch="CUDA graph of the whole forward" if args.graph else "eager",
+                 parallelism=f"dp{world}: {world} copies of the workload's requests, "
+                             "window-sharded across the ranks (LPT by tokens), "
+                             "rows kept on the rank that computed them")
+    return c
 
 
 def reference_arm(args, rank, world):
@@ -197,7 +207,8 @@ def reference_arm(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(ts) / len(ts),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": workload_config(args, world, lens_all, *layout_counts(cfg, lens_all)),
+            "config": workload_config(args, 1, lens_all, *layout_counts(cfg, lens_all),
+                                      impl="reference"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -211,15 +222,30 @@ def our_arm(args, rank, world, local_rank):
     from audio_encoder_aut_b200 import _lib as A
     from audio_encoder_aut_b200.encoder import Encoder
 
+    from audio_encoder_aut_b200 import shard as SH
+
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = S.WORKLOADS[args.workload]
-    lens = S.request_lengths(args.workload)
+    base = S.request_lengths(args.workload)
     w = S.weights(cfg)
-    feats = S.features(lens, seed=S.SEED_FEATURES + rank)
     enc = Encoder(cfg, w, local_rank)
+    # The whole job: `world` copies of the workload's requests (copy i with its
+    # own features), cut at window boundaries and assigned to the ranks by
+    # tokens; this rank encodes its shard as one packed batch.  One rank: the
+    # workload itself.
+    glens = base * world
+    shard = SH.assign(SH.pieces(glens, cfg.n_window_infer), world, enc.c)[rank]
+    copies = sorted({p.request // len(base) for p in shard})
+    feats_of = {i: S.features(base, seed=S.SEED_FEATURES + i) for i in copies}
+    lens = [p.frames for p in shard]
+    feats = np.zeros((len(shard), cfg.num_mel_bins, max(lens)), np.float32)
+    for j, p in enumerate(shard):
+        f = feats_of[p.request // len(base)][p.request % len(base)]
+        feats[j, :, :p.frames] = f[:, p.frame0:p.frame0 + p.frames]
     tpr, cu, T, nW, nch = enc.plan(lens)
     audio_s = sum(lens) / 100.0
+    job_audio_s = sum(glens) / 100.0
     fd = enc.features_to_device(feats)
     out = torch.empty((T, cfg.output_dim), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -263,8 +289,11 @@ def our_arm(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
     ms = total_ms / args.steps
-    value = world * audio_s * args.steps / (total_ms / 1e3)
-    tokens_s = world * T * args.steps / (total_ms / 1e3)
+    job_T = torch.tensor([T], dtype=torch.int64, device=dev)
+    if world > 1:
+        dist.all_reduce(job_T)
+    value = job_audio_s * args.steps / (total_ms / 1e3)
+    tokens_s = int(job_T.item()) * args.steps / (total_ms / 1e3)
     flops, gemm_flops = credited_flops(cfg, lens, cu)
     pk, pk_sus, hbm, pk_src = peaks()
 
@@ -324,7 +353,7 @@ def our_arm(args, rank, world, local_rank):
         t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_total = float(t.item())
-    e2e_value = world * audio_s * args.steps / (e2e_total / 1e3)
+    e2e_value = job_audio_s * args.steps / (e2e_total / 1e3)
     h_out = h_outs[0]
     del graphs
 
@@ -347,7 +376,7 @@ def our_arm(args, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(args, world, lens, T, nW, nch),
+            "config": workload_config(args, world, glens, int(job_T.item()), nW, nch),
             "tokens_per_s": tokens_s,
             "tflops": flops / (ms / 1e3) / 1e12,
             "pct_bf16_peak": 100 * flops / (ms / 1e3) / 1e12 / pk,
@@ -433,6 +462,13 @@ def sweep(args):
     assert enc.check() == 0
 
 
+def _spawned_rank(rank, world, port, argv):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.argv = [sys.argv[0]] + list(argv)
+    main()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -452,6 +488,15 @@ def main():
         return
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # Not under a launcher: start one process per GPU here.
+        import socket
+        import torch.multiprocessing as mp
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        mp.spawn(_spawned_rank, args=(args.gpus, port, sys.argv[1:]), nprocs=args.gpus, join=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -108,13 +108,14 @@ aut_status aut_plan(const aut_config *cfg, const int32_t *feature_lens, int32_t 
                     int32_t *tokens_per_request, int32_t *cu_seqlens,
                     int32_t *total_tokens, int32_t *num_windows, int32_t *num_chunks);
 
-/* Bytes of device workspace that aut_encode / aut_frontend / aut_encode_packed
- * need for a batch with these plan totals (from aut_plan).  Returns 0 for an
- * unsupported configuration. */
+/* No passage: a library helper.  Bytes of device workspace that aut_encode /
+ * aut_frontend / aut_encode_packed need for a batch with these plan totals
+ * (from aut_plan).  Returns 0 for an unsupported configuration. */
 size_t aut_workspace_bytes(const aut_config *cfg, int32_t total_tokens, int32_t num_windows,
                            int32_t num_chunks);
 
-/* Bytes of the device buffer aut_prepare_weights fills. */
+/* No passage: a library helper.  Bytes of the device buffer aut_prepare_weights
+ * fills. */
 size_t aut_prepared_bytes(const aut_config *cfg);
 
 /* One-time weight preparation (cubic.dev "Audio Encoder Component", Weight
@@ -232,8 +233,10 @@ aut_status aut_layernorm(const void *x, const void *gamma, const void *beta, voi
  * finer than bf16; values beyond +-65504 saturate), the operand of the fp16
  * o_proj GEMM.  The probabilities P enter the P V product as fp16 for head_dim
  * 64 (tensor-core path) and as two bf16 terms otherwise.  cu_seqlens: HOST int32
- * [num_windows + 1], every window at most 128 tokens.  workspace: device, at
- * least 4 * (num_windows + 1) bytes (the uploaded cu_seqlens). */
+ * [num_windows + 1], every window at most 128 tokens.  workspace: device, 4-byte
+ * aligned, at least 4 * (num_windows + 2) bytes: word 0 is the call's status
+ * word (aut_check(workspace) reads it after the stream is synchronised), the
+ * rest the uploaded cu_seqlens. */
 aut_status aut_window_attention(const void *qkv, void *out, int32_t T, int32_t d, int32_t heads,
                                 const int32_t *cu_seqlens, int32_t num_windows,
                                 void *workspace, size_t ws_bytes, aut_stream_t stream);
@@ -247,8 +250,13 @@ aut_status aut_window_attention(const void *qkv, void *out, int32_t T, int32_t d
  * its scratch (the uploaded cu_seqlens) in a file-scope device array of the
  * library instead of a caller workspace.
  * Limits and behaviour:
- *   - num_windows at most 32767 (128 KiB of scratch); larger returns
- *     AUT_ERR_WORKSPACE before anything is launched.
+ *   - num_windows at most 32766 (128 KiB of scratch: one status word and
+ *     cu_seqlens); larger returns AUT_ERR_WORKSPACE before anything is
+ *     launched.
+ *   - Device-side faults (a pipeline wait that ran out of time) go to a status
+ *     word in the same array, cleared by every call; aut_check_status_word(NULL)
+ *     reads and clears it for the current device after the stream is
+ *     synchronised.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.
@@ -261,16 +269,64 @@ aut_status aut_window_attention_noalloc(const void *qkv, void *out, int32_t T, i
                                         int32_t heads, const int32_t *cu_seqlens,
                                         int32_t num_windows, aut_stream_t stream);
 
-/* Reads and clears the device status word of a workspace used by aut_encode /
+/* Log-mel front end (cubic.dev "Audio Encoder Component", Feature Extraction
+ * Pipeline: 16 kHz mono audio -> 128-bin mel spectrogram; m-star.org
+ * aut_encoder page, module docstring: Whisper-style log-mel, 100 frames/s).
+ * The steps the pages leave open follow Whisper's recipe: 400-sample periodic
+ * Hann frames every 160 samples, centred, the signal reflected by 200 samples
+ * at both ends; power of the 400-point DFT; 128 Slaney mel filters of unit
+ * area over 0..8000 Hz; log10 of max(energy, 1e-10); the transform's last
+ * frame dropped, so n samples give n / 160 frames; per request, values raised
+ * to at least (that request's maximum - 8); then (x + 4) / 4.
+ * waveform: device fp32 [n_req, S_max] (request r's first sample_lens[r]
+ * samples are used).  sample_lens: HOST int32 [n_req], each 0 or in
+ * (200, S_max].  features: device bf16 [n_req, 128, T_max], T_max at least the
+ * longest request's frames; written whole (zeros past each request's frames),
+ * ready for aut_encode.  feature_lens: HOST int32 [n_req] out (may be NULL):
+ * sample_lens[r] / 160.  workspace: device, 256-byte aligned, at least
+ * aut_logmel_workspace_bytes(n_req, T_max).  Argument errors return before any
+ * launch; asynchronous on `stream`. */
+aut_status aut_logmel(const void *waveform, int64_t S_max, const int32_t *sample_lens,
+                      int32_t n_req, void *features, int32_t T_max, int32_t *feature_lens,
+                      void *workspace, size_t ws_bytes, aut_stream_t stream);
+
+/* No passage: a library helper.  Bytes of device workspace aut_logmel needs. */
+size_t aut_logmel_workspace_bytes(int32_t n_req, int32_t T_max);
+
+/* Audio injection into the decoder's input (cubic.dev "Audio Encoder
+ * Component", Audio Injection Logic: the encoder's features replace the
+ * embeddings at the <|audio_pad|> placeholder positions).  The j-th position
+ * (in sequence order) whose token id equals audio_pad_id receives row j of
+ * `audio`; every other row of `embeds` is left as it is.
+ * embeds: device bf16 [L, D], updated in place (8-byte aligned); token_ids:
+ * device int32 [L]; audio: device fp32 [T, D] (16-byte aligned), e.g. the
+ * output of aut_encode (rows in packed order), rounded to bf16 (nearest even)
+ * on the way in.  workspace: device, 256-byte aligned, at least
+ * aut_inject_workspace_bytes(L).  The number of placeholders is counted on the
+ * device: if it is not T, aut_check(workspace) reports AUT_ERR_INVALID_ARG
+ * after the stream is synchronised and no row past T is read (placeholders
+ * beyond the T-th keep their embeddings).  Asynchronous on `stream`. */
+aut_status aut_inject_audio(void *embeds, const int32_t *token_ids, int32_t L,
+                            int32_t audio_pad_id, const void *audio, int32_t T, int32_t D,
+                            void *workspace, size_t ws_bytes, aut_stream_t stream);
+
+/* No passage: a library helper.  Bytes of device workspace aut_inject_audio needs. */
+size_t aut_inject_workspace_bytes(int32_t L);
+
+/* No passage: a library helper.  Reads and clears the device status word of a
+ * workspace used by aut_window_attention or by aut_encode /
  * aut_frontend / aut_encode_packed (synchronous: call after the stream is
  * synchronised).  Each of those calls clears the word when it starts, so this
  * reports the first device-side fault of the latest call on the workspace. */
 aut_status aut_check(void *workspace);
 
-/* Reads and clears a status word given to aut_linear (synchronous). */
+/* No passage: a library helper.  Reads and clears a status word given to
+ * aut_linear (synchronous).  NULL
+ * selects the status word of aut_window_attention_noalloc on the current
+ * device. */
 aut_status aut_check_status_word(int32_t *status);
 
-/* Static text for a status code. */
+/* No passage: a library helper.  Static text for a status code. */
 const char *aut_status_string(aut_status status);
 
 #ifdef __cplusplus

@@ -10,3 +10,4 @@ say the encoder computes, in fp64 (or fp32 for the large workloads), sharing no
 code, tables or constants with the CUDA path.
 """
 from .aut_oracle import *  # noqa: F401,F403
+from . import inject, logmel  # noqa: F401

@@ -241,3 +241,34 @@ def test_pipelined_host_stream_matches_eager_bit_exact():
     torch.cuda.synchronize()
     for b, h in zip(batches[3:], host_out2):
         assert np.array_equal(h.numpy(), run(enc, b, lens))
+
+
+@pytest.mark.parametrize("name,lens,max_frames,world", [
+    ("omni_16req", [1734, 90, 610, 2999, 333, 1201], 1600, 3),
+    ("tiny", [1234, 90, 610, 0, 333], 400, 4),
+])
+def test_sharded_pieces_reassemble_bit_exact(name, lens, max_frames, world):
+    """The multi-GPU split on one device: a `world`-rank plan of window-aligned
+    pieces (long requests cut at window boundaries), every rank's pieces
+    encoded as its own packed batch through aut_encode, reassembled into
+    packed order, equals the unsharded forward bit for bit (window isolation,
+    aut_encoder page module docstring; openarchlab 1A, section 4)."""
+    from audio_encoder_aut_b200 import shard as SH
+    cfg, w, enc = encoder(name)
+    feats = S.features(lens)
+    whole = run(enc, feats, lens)
+    shards = SH.assign(SH.pieces(lens, cfg.n_window_infer, max_frames), world, enc.c)
+    assert sum(len(s) > 0 for s in shards) >= 2
+    fd = enc.features_to_device(feats)
+    outs = []
+    for s in shards:
+        if s:
+            o = enc.encode(SH.shard_features(fd, s), [p.frames for p in s])
+            torch.cuda.synchronize()
+            assert enc.check() == A.AUT_OK
+            outs.append(o.cpu().numpy())
+        else:
+            outs.append(np.zeros((0, cfg.output_dim), np.float32))
+    got = SH.reassemble(enc.c, shards, outs)
+    assert got.shape == whole.shape
+    assert np.array_equal(got, whole)

@@ -175,23 +175,27 @@ def test_window_attention_matches_oracle(heads, hd, lens):
     assert_f16_output_close(o, ref, "window attention", atol=2e-4 * vmax)
 
 
-def test_pipeline_wait_timeout_returns_status_and_gpu_stays_usable():
+@pytest.mark.parametrize("mode", [0, A.LINEAR_SINGLE_CTA], ids=["cta_pair", "single_cta"])
+def test_pipeline_wait_timeout_returns_status_and_gpu_stays_usable(mode):
     """A GEMM whose first block never receives its first operand tile: the
     consumer's bounded wait runs out, the kernel records AUT_ERR_TIMEOUT and
-    returns; the next launch on the same context works."""
+    returns; the next launch on the same context works.  In CTA-pair mode the
+    skipped stage is the even CTA's, so the odd CTA's wait for that stage to be
+    armed runs out as well, and the pair still leaves through its cluster
+    barrier."""
     M, N, K = 256, 128, 128
     x = _dev(_rand((M, K), 1), torch.bfloat16)
     w = _dev(_rand((N, K), 2, 0.05), torch.bfloat16)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     st = A.aut_linear(x.data_ptr(), w.data_ptr(), None, y.data_ptr(), M, N, K, A.EPI_BF16,
-                      status.data_ptr(), 200, A.LINEAR_FAULT_INJECT, _stream())
+                      status.data_ptr(), 200, A.LINEAR_FAULT_INJECT | mode, _stream())
     assert st == A.AUT_OK
     torch.cuda.synchronize()
     assert A.aut_check_status_word(status.data_ptr()) == A.AUT_ERR_TIMEOUT
     assert int(status.item()) == 0  # cleared by the check
     st = A.aut_linear(x.data_ptr(), w.data_ptr(), None, y.data_ptr(), M, N, K, A.EPI_BF16,
-                      status.data_ptr(), 0, 0, _stream())
+                      status.data_ptr(), 0, mode, _stream())
     torch.cuda.synchronize()
     assert st == A.AUT_OK and A.aut_check_status_word(status.data_ptr()) == A.AUT_OK
     ref = x.float().cpu().numpy().astype(np.float64) @ w.float().cpu().numpy().astype(np.float64).T

@@ -12,7 +12,14 @@ import torch.multiprocessing as mp
 
 import aut_synth as S
 import oracle as O
+from audio_encoder_aut_b200 import _lib as A
 from audio_encoder_aut_b200 import shard as SH
+
+CFG = A.make_config(S.TINY)
+
+
+def _tok(frames):
+    return SH.frame_tokens(CFG, [frames])[0]
 
 
 def test_pieces_and_assignment_cover_the_batch():
@@ -26,13 +33,13 @@ def test_pieces_and_assignment_cover_the_batch():
             assert f0 == covered and f0 % 800 == 0
             covered += nf
         assert covered == n
-    shards = SH.assign(ps, 3)
+    shards = SH.assign(ps, 3, CFG)
     assert sorted(p for s in shards for p in s) == sorted(ps)
-    loads = [sum(SH._tokens(p.frames) for p in s) for s in shards]
-    assert max(loads) - min(loads) <= max(SH._tokens(p.frames) for p in ps)
+    loads = [sum(_tok(p.frames) for p in s) for s in shards]
+    assert max(loads) - min(loads) <= max(_tok(p.frames) for p in ps)
     # token counts of the pieces add up to the requests' token counts
     for r, n in enumerate(lens):
-        assert sum(SH._tokens(p.frames) for p in ps if p.request == r) == \
+        assert sum(_tok(p.frames) for p in ps if p.request == r) == \
             O.tokens_for_frames(S.TINY, n)
 
 
@@ -49,20 +56,19 @@ def _rank_main(rank, world, port, lens, result_path):
         cfg = S.TINY
         w = S.weights(cfg, conv_scale=10.0)
         feats = S.features(lens)
-        shards = SH.assign(SH.pieces(lens, cfg.n_window_infer, max_frames=400), world)
+        shards = SH.assign(SH.pieces(lens, cfg.n_window_infer, max_frames=400), world,
+                           A.make_config(cfg))
         mine = shards[rank]
         if mine:
             sub_lens = [p.frames for p in mine]
-            sub = np.zeros((len(mine), feats.shape[1], max(sub_lens)), np.float32)
-            for i, p in enumerate(mine):
-                sub[i, :, :p.frames] = feats[p.request, :, p.frame0:p.frame0 + p.frames]
+            sub = SH.shard_features(feats, mine)
             out, _ = O.forward(cfg, w, sub, sub_lens)
         else:
             out = np.zeros((0, cfg.output_dim))
         gathered = [None] * world
         dist.all_gather_object(gathered, out)
         if rank == 0:
-            got = SH.reassemble(lens, shards, gathered)
+            got = SH.reassemble(A.make_config(cfg), shards, gathered)
             ref, _ = O.forward(cfg, w, feats, lens)
             np.save(result_path, np.stack([np.abs(got - ref).max(), float(got.shape[0] == ref.shape[0])]))
     finally:
@@ -99,23 +105,23 @@ def test_shard_planner_properties_random():
                 assert f0 == covered and f0 % nwi == 0 and nf > 0
                 covered += nf
             assert covered == n
-            assert sum(SH._tokens(p.frames) for p in ps if p.request == r) == \
+            assert sum(_tok(p.frames) for p in ps if p.request == r) == \
                 O.tokens_for_frames(S.TINY, n)
-        shards = SH.assign(ps, world)
+        shards = SH.assign(ps, world, CFG)
         assert len(shards) == world
         assert sorted(p for s in shards for p in s) == sorted(ps)
         if ps:
-            loads = [sum(SH._tokens(p.frames) for p in s) for s in shards]
-            assert max(loads) - min(loads) <= max(SH._tokens(p.frames) for p in ps)
+            loads = [sum(_tok(p.frames) for p in s) for s in shards]
+            assert max(loads) - min(loads) <= max(_tok(p.frames) for p in ps)
         # each rank's "output" rows hold (request, token index within the request)
         outputs = []
         for s in shards:
             rows = []
             for p in s:
-                t0 = SH._tokens(p.frame0)
-                rows += [(p.request, t0 + i) for i in range(SH._tokens(p.frames))]
+                t0 = _tok(p.frame0)
+                rows += [(p.request, t0 + i) for i in range(_tok(p.frames))]
             outputs.append(np.array(rows, dtype=np.int64).reshape(-1, 2))
-        got = SH.reassemble(lens, shards, outputs)
+        got = SH.reassemble(CFG, shards, outputs)
         want = [(r, i) for r, n in enumerate(lens) for i in range(O.tokens_for_frames(S.TINY, n))]
         if want:
             assert got.tolist() == [list(w) for w in want]

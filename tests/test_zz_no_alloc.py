@@ -12,16 +12,22 @@ from audio_encoder_aut_b200 import _lib as A
 
 
 def test_noalloc_rejects_too_many_windows_before_any_launch():
-    # Checked on the host before anything touches a GPU (none is needed).
-    assert A.aut_window_attention_noalloc(1024, 1024, 0, 64, 4, [0] * 32770, 0) == \
+    # Checked on the host before anything touches a GPU (none is needed): the
+    # array holds a status word and at most 32767 cu_seqlens entries.
+    assert A.aut_window_attention_noalloc(1024, 1024, 0, 64, 4, [0] * 32768, 0) == \
         A.AUT_ERR_WORKSPACE
 
 
 @pytest.mark.gpu
 def test_noalloc_attention_matches_workspace_attention_on_two_calls():
+    """Calls in a row, each checked against the workspace entry point; the
+    third has a single window after one with six, so it must ignore the stale
+    cu_seqlens entries the earlier call left in the shared array.  After every
+    call the status word of the allocation-free entry reads OK."""
     torch = pytest.importorskip("torch")
     st = torch.cuda.current_stream().cuda_stream
-    cases = [(20, 64, [104, 104, 1, 17, 128, 50]), (4, 16, [26, 5, 26, 26, 3])]
+    cases = [(20, 64, [104, 104, 1, 17, 128, 50]), (4, 16, [26, 5, 26, 26, 3]),
+             (20, 64, [77])]
     for call, (heads, hd, lens) in enumerate(cases):
         d = heads * hd
         cu = [0]
@@ -46,3 +52,5 @@ def test_noalloc_attention_matches_workspace_attention_on_two_calls():
         assert np.isfinite(g).all()
         np.testing.assert_allclose(g, r, rtol=1e-4, atol=1e-4 * np.abs(r).max())
         assert np.array_equal(g, r)
+        assert A.aut_check_status_word(None) == A.AUT_OK
+        assert A.aut_check(ws.data_ptr()) == A.AUT_OK
