@@ -86,6 +86,9 @@ _SIGNATURES = {
                                 c_float, c_void_p]),
     "aut_window_attention": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                        POINTER(c_int32), c_int32, c_void_p, c_size_t, c_void_p]),
+    "aut_window_attention_ex": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32,
+                                          POINTER(c_int32), c_int32, c_void_p, c_size_t, c_int32,
+                                          c_int32, c_void_p]),
     "aut_window_attention_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                                POINTER(c_int32), c_int32, c_void_p]),
     "aut_logmel": (c_int32, [c_void_p, ctypes.c_int64, POINTER(c_int32), c_int32, c_void_p,
@@ -229,6 +232,17 @@ def aut_window_attention(qkv: int, out: int, T: int, d: int, heads: int, cu_seql
                          workspace: int, ws_bytes: int, stream: int) -> int:
     return lib().aut_window_attention(qkv, out, T, d, heads, _i32(cu_seqlens),
                                       len(cu_seqlens) - 1, workspace, ws_bytes, stream)
+
+
+def aut_window_attention_ex(qkv: int, out: int, T: int, d: int, heads: int, cu_seqlens,
+                            workspace: int, ws_bytes: int, timeout_ms: int, flags: int,
+                            stream: int) -> int:
+    return lib().aut_window_attention_ex(qkv, out, T, d, heads, _i32(cu_seqlens),
+                                         len(cu_seqlens) - 1, workspace, ws_bytes, timeout_ms,
+                                         flags, stream)
+
+
+ATTN_FAULT_INJECT = 1
 
 
 def aut_window_attention_noalloc(qkv: int, out: int, T: int, d: int, heads: int, cu_seqlens,

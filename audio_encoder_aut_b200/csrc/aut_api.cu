@@ -495,6 +495,16 @@ extern "C" aut_status aut_window_attention(const void *qkv, void *out, int32_t T
                                            int32_t heads, const int32_t *cu_seqlens,
                                            int32_t num_windows, void *workspace, size_t ws_bytes,
                                            aut_stream_t stream) {
+    return aut_window_attention_ex(qkv, out, T, d, heads, cu_seqlens, num_windows, workspace,
+                                   ws_bytes, 0, 0, stream);
+}
+
+extern "C" aut_status aut_window_attention_ex(const void *qkv, void *out, int32_t T, int32_t d,
+                                              int32_t heads, const int32_t *cu_seqlens,
+                                              int32_t num_windows, void *workspace,
+                                              size_t ws_bytes, int32_t timeout_ms, int32_t flags,
+                                              aut_stream_t stream) {
+    if (timeout_ms < 0 || (flags & ~AUT_ATTN_FAULT_INJECT)) return AUT_ERR_INVALID_ARG;
     if (T < 0 || d <= 0 || heads <= 0 || d % heads || num_windows < 0 || !cu_seqlens)
         return AUT_ERR_INVALID_ARG;
     const int hd = d / heads;
@@ -516,8 +526,11 @@ extern "C" aut_status aut_window_attention(const void *qkv, void *out, int32_t T
     words.insert(words.end(), cu_seqlens, cu_seqlens + num_windows + 1);
     int32_t *ws = static_cast<int32_t *>(workspace);
     AUT_TRY(cuda_status(launch_upload(words.data(), words.size(), ws, st)));
-    return cuda_status(
-        launch_window_attention(qkv, out, ws + 1, num_windows, d, heads, st, T, ws));
+    const bool fault = (flags & AUT_ATTN_FAULT_INJECT) != 0;
+    if (fault && !window_attention_uses_tc(d, heads, T)) return AUT_ERR_UNSUPPORTED;
+    return cuda_status(launch_window_attention(
+        qkv, out, ws + 1, num_windows, d, heads, st, T, ws, false,
+        timeout_ms ? (unsigned long long)timeout_ms * 1000000ull : 0ull, fault ? 1 : 0));
 }
 
 extern "C" aut_status aut_check_status_word(int32_t *status) {

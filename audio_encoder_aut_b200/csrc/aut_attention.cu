@@ -6,37 +6,39 @@
 // segment).  A window has at most 128 tokens, so one (window, head) is one
 // 128-row tile and the softmax is exact in one pass over the tile.
 //
-// The kernel is persistent (two CTAs per SM) and walks the (window, head)
+// The kernel is persistent (one CTA per SM) and walks the (window, head)
 // tiles with a grid stride.  Warp roles:
 //   warp 0     TMA producer: Q, K, V tiles [128 x 64] bf16 (128-byte swizzle)
 //              from qkv [T, 3d] into a ring of kStages stages; rows past the
 //              window's end are the next window's rows (or zero past T) and
 //              are masked below
-//   warp 1     MMA issuer:  S = Q K^T  (M = 128, N = window length rounded up
-//              to 16, K = 64) into TMEM columns 0..127; once P is ready,
-//              O = P V (M = 128, N = 64, K = window length rounded up to 16,
-//              fp16 inputs, V read MN-major) into one of two O buffers (TMEM
-//              columns 128..191 and 192..255), so tile k's softmax overlaps
-//              the O product of tile k - 1
-//   warps 2-9  softmax and epilogue, two warps per TMEM lane quadrant, each
-//              over half of the keys: row max (exchanged between the two
-//              halves), p = exp2(s log2(e) / sqrt(64) - max log2(e) / sqrt(64)) written to
-//              shared memory as fp16 (P lies in [0, 1]; fp16 keeps 11
-//              significant bits, 8x finer than bf16) in the swizzled K-major
-//              layout the MMA reads, over the Q and K tiles the first MMA no
-//              longer needs; V converted in place to fp16 (saturating: bf16
-//              values beyond fp16's range clamp to +-65504) unless the qkv
-//              GEMM already wrote it as fp16 (v_f16); then O / rowsum
-//              written as fp16 [T, d] (11 significant bits for the o_proj GEMM,
-//              which runs on fp16 operands; rows past the window's end are not
+//   warp 1     MMA issuer: S = Q K^T (M = 128, N = the window length rounded
+//              up to 16, K = 64) into the S buffer of the tile's softmax
+//              group; once that group has written P, O = P V (M = 128, N = 64,
+//              K = window length rounded up to 16, fp16 inputs, V read
+//              MN-major) into one of the group's two O buffers, then S of the
+//              group's next tile
+//   warps 2-9  two softmax groups of four warps (one per TMEM lane quadrant);
+//              group g takes the CTA's tiles g, g + 2, g + 4, ...  Every
+//              thread owns one query row and all of its keys, so the row max
+//              and sum need no exchange between threads: max over the row,
+//              p = exp2(s log2(e) / sqrt(64) - max log2(e) / sqrt(64)) written
+//              as fp16 (P lies in [0, 1]; 11 significant bits, 8x finer than
+//              bf16) in the swizzled K-major layout the MMA reads, over the Q
+//              and K tiles the S product no longer needs; V converted in place
+//              to fp16 (saturating) unless the qkv GEMM already wrote it as fp16
+//              (v_f16); then, while the tensor cores compute this tile's O and
+//              the group's next S, O / rowsum of the group's previous tile
+//              written as fp16 [T, d] (rows past the window's end are not
 //              written)
-// The producer runs up to kStages tiles ahead, so the loads of the next tiles
-// overlap the softmax and the stores of this one; the second CTA on the SM
-// fills the gaps of the first.
+// While one group runs its softmax the other's S and O products run on the
+// tensor cores, and the producer stays up to kStages tiles ahead.
 //
-// Two TMEM users never share an SM between kernels of the forward: this
-// kernel's shared memory (about 100 KB) and the GEMM's (about 197 KB) exceed
-// the SM's 228 KB together, so a CTA launched early by programmatic dependent
+// Tensor memory (512 columns): S buffers of the two groups at 0 and 128; O
+// buffers (64 columns) at 256 + 64 (2 g + j), j alternating over the group's
+// tiles.  Two TMEM users never share an SM between kernels of the forward:
+// this kernel's shared memory (about 197 KB) leaves no room for a GEMM CTA
+// (about 197 KB either), so a CTA launched early by programmatic dependent
 // launch cannot hold TMEM columns that a CTA of the previous kernel still needs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -55,19 +57,17 @@ using bf16 = __nv_bfloat16;
 constexpr int kTile = 128;                   // query / key rows per tile
 constexpr int kHd = 64;                      // head dim (one 128-byte swizzle row)
 constexpr int kTileBytes = kTile * kHd * 2;  // 16 KiB
-constexpr int kStages = 2;
+constexpr int kStages = 4;
 constexpr int kStageBytes = 3 * kTileBytes;  // Q | K | V; P (fp16, 128 x 128) overwrites Q | K
-constexpr int kOffRed = kStages * kStageBytes;  // row max and sum of the two key halves
-constexpr int kOffBar = kOffRed + 2 * 2 * kTile * 4;
-// full[kStages], empty[kStages], s_full, p_full, o_full[2], o_empty[2], mma_done
-constexpr int kNumBars = 2 * kStages + 2 + 4 + 1;
+constexpr int kGroups = 2;                   // softmax groups (four warps each)
+constexpr int kOffBar = kStages * kStageBytes;
+// full[kStages], empty[kStages], s_full[2], p_full[2], o_full[4], o_empty[4], mma_done
+constexpr int kNumBars = 2 * kStages + 2 * kGroups + 4 + 4 + 1;
 constexpr int kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
-constexpr int kComputeWarps = 8;
+constexpr int kComputeWarps = 4 * kGroups;
 constexpr int kThreads = 64 + 32 * kComputeWarps;
-constexpr int kCtasPerSm = 2;
-constexpr uint32_t kTmemCols = 256;  // S: 0..127, O: two buffers at 128..191 and 192..255
-constexpr uint32_t kColO = 128;
-constexpr unsigned long long kTimeoutNs = 4000ull * 1000ull * 1000ull;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;  // O buffer b (0..3) at kColO + 64 b
 
 // kind::f16 with fp16 A and B, fp32 accumulate, A K-major, B MN-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
@@ -79,31 +79,6 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
 __device__ __forceinline__ uint32_t p_chunk_offset(int r, int chunk) {
     const int atom = chunk >> 3, c = chunk & 7;
     return (uint32_t)(atom * kTileBytes + r * 128 + ((c ^ (r & 7)) << 4));
-}
-
-// Named barrier ID over the 64 threads of two warps that also ORs their `fail`
-// flags: both warps get the same answer, so they leave a loop together.
-template <int ID>
-__device__ __forceinline__ bool sync_any_64(bool fail) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, 64, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(r)
-        : "r"((uint32_t)fail), "n"(ID)
-        : "memory");
-    return r != 0;
-}
-// The barrier of lane quadrant `quad` (ids 1-4; 0 is __syncthreads).
-__device__ __forceinline__ bool quad_sync_any(int quad, bool fail) {
-    switch (quad) {
-        case 0: return sync_any_64<1>(fail);
-        case 1: return sync_any_64<2>(fail);
-        case 2: return sync_any_64<3>(fail);
-        default: return sync_any_64<4>(fail);
-    }
 }
 
 __device__ __forceinline__ void signal_abort(int *status, volatile int *abort) {
@@ -118,21 +93,20 @@ __device__ __forceinline__ void window_of(const int *cu, int w, int *s0, int *le
     *n16 = max(1, (*len + 15) >> 4);
 }
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
+__global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_qkv, __half *__restrict__ out, const int *__restrict__ cu,
-    int n_windows, int heads, int d, float scale_log2e, int *status, int v_f16) {
+    int n_windows, int heads, int d, float scale_log2e, int *status, int v_f16,
+    unsigned long long lim, int fault_inject) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *red_max = reinterpret_cast<float *>(sm + kOffRed);  // [2 halves][128 rows]
-    float *red_sum = red_max + 2 * kTile;
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + kOffBar);
     uint64_t *empty = full + kStages;
-    uint64_t *s_full = empty + kStages;  // S in TMEM
-    uint64_t *p_full = s_full + 1;       // P and fp16 V in shared memory, S read
-    uint64_t *o_full = p_full + 1;       // [2] O buffer in TMEM
-    uint64_t *o_empty = o_full + 2;      // [2] O buffer read out of TMEM
-    uint64_t *mma_done = o_empty + 2;
+    uint64_t *s_full = empty + kStages;  // [2] S of the group's tile in TMEM
+    uint64_t *p_full = s_full + kGroups; // [2] P (and fp16 V) in shared memory, S read
+    uint64_t *o_full = p_full + kGroups; // [4] O buffer complete
+    uint64_t *o_empty = o_full + 4;      // [4] O buffer read out of TMEM
+    uint64_t *mma_done = o_empty + 4;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(mma_done + 1);
     int *abort_flag = reinterpret_cast<int *>(tslot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,11 +117,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, kComputeWarps);
-        for (int b = 0; b < 2; ++b) {
+        for (int g = 0; g < kGroups; ++g) {
+            mbar_init(s_full + g, 1);
+            mbar_init(p_full + g, 4);
+        }
+        for (int b = 0; b < 4; ++b) {
             mbar_init(o_full + b, 1);
-            mbar_init(o_empty + b, kComputeWarps);
+            mbar_init(o_empty + b, 4);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -165,21 +141,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
     volatile int *abort_v = abort_flag;
     pdl_wait();
     const int n_tiles = n_windows * heads;
+    // This CTA's tiles: blockIdx.x + k gridDim.x for k < n_local.
+    const int n_local = blockIdx.x < n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    auto tile_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer --
             uint32_t issued = 0, parity = 0;
             bool ok = true;
-            int k = 0;
-            for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++k) {
-                const int w = t / heads, h = t - w * heads;
+            for (int k = 0; k < n_local; ++k) {
+                const int t = tile_of(k), w = t / heads, h = t - w * heads;
                 const int s = k % kStages;
                 const uint32_t use = (uint32_t)(k / kStages);
-                if (k >= kStages && !mbar_wait(empty + s, (use - 1) & 1u, abort_v, kTimeoutNs)) {
+                if (k >= kStages && !mbar_wait(empty + s, (use - 1) & 1u, abort_v, lim)) {
                     ok = false;
                     break;
                 }
+                if (fault_inject && blockIdx.x == 0 && k == 0) continue;  // never filled
                 uint8_t *st = sm + s * kStageBytes;
                 const int s0 = cu[w];
                 mbar_arrive_expect_tx(full + s, kStageBytes);
@@ -190,53 +169,46 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
                 parity = (parity & ~(1u << s)) | ((use & 1u) << s);
             }
             if (!ok) signal_abort(status, abort_v);
-            // The last load issued on every stage has landed before the block may exit.
-            for (int s = 0; s < kStages; ++s)
-                if (issued >> s & 1u) mbar_wait(full + s, parity >> s & 1u, nullptr, kTimeoutNs);
+            // The last load issued on every stage has landed before the block
+            // may exit (one shared time limit for all of them).
+            const uint64_t t0 = global_timer_ns();
+            for (int s = 0; s < kStages; ++s) {
+                const uint64_t used = global_timer_ns() - t0;
+                if ((issued >> s & 1u) && used < lim)
+                    mbar_wait(full + s, parity >> s & 1u, nullptr, lim - used);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // -------------------------------------------------- MMA issuer --
             constexpr uint32_t idesc_o = idesc_f16_f32_bmn(kTile, kHd);
             bool ok = true;
-            // S of local tile kk (global tile t): N = the window's keys rounded up
-            // to 16.  Needs the tile's loads and a free S buffer.
-            auto issue_s = [&](int kk, int t) -> bool {
+            // S of local tile k into its group's S buffer.
+            auto issue_s = [&](int k) -> bool {
                 int s0, len, n16;
-                window_of(cu, t / heads, &s0, &len, &n16);
-                const int s = kk % kStages;
-                if (!mbar_wait(full + s, (uint32_t)(kk / kStages) & 1u, abort_v, kTimeoutNs))
-                    return false;
+                window_of(cu, tile_of(k) / heads, &s0, &len, &n16);
+                const int s = k % kStages;
+                if (!mbar_wait(full + s, (uint32_t)(k / kStages) & 1u, abort_v, lim)) return false;
                 tc_fence_after();
                 uint8_t *st = sm + s * kStageBytes;
                 const uint32_t idesc_s = idesc_bf16_f32(kTile, 16 * n16);
 #pragma unroll
                 for (int q = 0; q < kHd / 16; ++q)
-                    tc_mma_bf16(tmem, smem_desc_sw128(st) + 2 * q,
+                    tc_mma_bf16(tmem + (k & 1) * kTile, smem_desc_sw128(st) + 2 * q,
                                 smem_desc_sw128(st + kTileBytes) + 2 * q, idesc_s, q > 0);
-                tc_commit(s_full);
+                tc_commit(s_full + (k & 1));
                 return true;
             };
-            int k = 0;
-            if (blockIdx.x < n_tiles) ok = issue_s(0, blockIdx.x);
-            for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++k) {
+            for (int k = 0; ok && k < n_local && k < kGroups; ++k) ok = issue_s(k);
+            for (int k = 0; ok && k < n_local; ++k) {
                 int s0, len, n16;
-                window_of(cu, t / heads, &s0, &len, &n16);
-                const int s = k % kStages;
-                uint8_t *st = sm + s * kStageBytes;
-                // P of tile k is in shared memory and S has been read: S of the
-                // next tile goes first (the softmax waits for it), then O of this.
-                if (!mbar_wait(p_full, k & 1u, abort_v, kTimeoutNs)) {
-                    ok = false;
-                    break;
-                }
-                if (t + (int)gridDim.x < n_tiles && !issue_s(k + 1, t + gridDim.x)) {
-                    ok = false;
-                    break;
-                }
-                // O buffer k & 1 was last drained by the epilogue of tile k - 2.
-                const int ob = k & 1;
-                if (k >= 2 && !mbar_wait(o_empty + ob, ((k - 2) >> 1) & 1u, abort_v, kTimeoutNs)) {
+                window_of(cu, tile_of(k) / heads, &s0, &len, &n16);
+                const int g = k & 1, ob = 2 * g + ((k >> 1) & 1);
+                uint8_t *st = sm + (k % kStages) * kStageBytes;
+                // P of tile k is in shared memory (and S has been read); the O
+                // buffer was last drained by the epilogue of the group's tile k - 4.
+                if (!mbar_wait(p_full + g, (uint32_t)(k >> 1) & 1u, abort_v, lim) ||
+                    (k >= 4 && !mbar_wait(o_empty + ob, (uint32_t)((k >> 2) - 1) & 1u, abort_v, lim))) {
                     ok = false;
                     break;
                 }
@@ -248,110 +220,99 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
                                 smem_desc_sw128_mn(st + 2 * kTileBytes + j * 16 * 128), idesc_o,
                                 j > 0);
                 tc_commit(o_full + ob);
-                tc_commit(empty + s);  // Q | K (now P) and V free once O is done
+                tc_commit(empty + k % kStages);  // Q | K (now P) and V free once O is done
+                // The group's next S reuses the S buffer this tile's softmax has read.
+                if (k + kGroups < n_local && !issue_s(k + kGroups)) ok = false;
             }
             if (!ok) signal_abort(status, abort_v);
             // Every MMA this thread issued has completed before TMEM is released.
             tc_commit(mma_done);
-            mbar_wait(mma_done, 0, nullptr, kTimeoutNs);
+            mbar_wait(mma_done, 0, nullptr, lim);
         }
     } else {
         // --------------------------------------------- softmax, epilogue --
-        // Tile k's softmax runs while the tensor cores finish O of tile k - 1
-        // (two O buffers); tile k - 1's epilogue follows, by which time S of
-        // tile k + 1 is being computed.  The two warps of a lane quadrant meet at
-        // a named barrier that also ORs their failure flags, so both leave the
-        // loop together after a time-out.
-        const int cw = warp - 2, ctid = threadIdx.x - 64;
+        const int cw = warp - 2, g = cw >> 2;
         const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
-        const int half = cw >> 2;   // keys [64 half, 64 half + 64); O columns [32 half, + 32)
         const int row = quad * 32 + lane;
+        const int gtid = (cw & 3) * 32 + lane;  // 0 .. 127 inside the group
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
         bool fail = false;
-        // Epilogue of local tile kk (global tile t): O / rowsum to fp16 rows.
-        auto epilogue = [&](int kk, int t, float inv) {
-            const int w = t / heads, h = t - w * heads;
+        // Epilogue of local tile kk: O / rowsum to fp16 rows.
+        auto epilogue = [&](int kk, float inv) {
+            const int t = tile_of(kk), w = t / heads, h = t - w * heads;
             int s0, len, n16;
             window_of(cu, w, &s0, &len, &n16);
-            const int ob = kk & 1;
-            fail = fail || !mbar_wait(o_full + ob, (kk >> 1) & 1u, abort_v, kTimeoutNs);
-            fail = __any_sync(0xffffffffu, fail);
+            const int ob = 2 * g + ((kk >> 1) & 1);
+            fail = fail || !mbar_wait_warp(o_full + ob, (uint32_t)(kk >> 2) & 1u, abort_v, lim);
             if (fail) return;
             tc_fence_after();
             const bool active = quad * 32 < len;
-            float o[32];
+            float o[2][32];
             if (active) {
-                tmem_ld32(trow + kColO + ob * kHd + half * 32, o);
+                tmem_ld32(trow + kColO + ob * kHd, o[0]);
+                tmem_ld32(trow + kColO + ob * kHd + 32, o[1]);
                 tc_wait_ld();
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(o_empty + ob);
             if (active && row < len) {
-                __half *dst = out + (size_t)(s0 + row) * d + h * kHd + half * 32;
+                __half *dst = out + (size_t)(s0 + row) * d + h * kHd;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 8; ++q) {
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        pk[e] = pack_f16x2_sat(o[q * 8 + 2 * e] * inv, o[q * 8 + 2 * e + 1] * inv);
+                        pk[e] = pack_f16x2_sat(o[q >> 2][(q & 3) * 8 + 2 * e] * inv,
+                                               o[q >> 2][(q & 3) * 8 + 2 * e + 1] * inv);
                     *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
         };
-        int k = 0, prev_t = -1;
+        int prev_k = -1;
         float prev_inv = 0.f;
-        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++k) {
+        for (int k = g; k < n_local; k += kGroups) {
             int s0, len, n16;
-            window_of(cu, t / heads, &s0, &len, &n16);
+            window_of(cu, tile_of(k) / heads, &s0, &len, &n16);
             const int s = k % kStages;
-            const uint32_t use = (uint32_t)(k / kStages);
             uint8_t *st = sm + s * kStageBytes;
+            const uint32_t t_s = trow + g * kTile;
             const bool active = quad * 32 < len;  // warp-uniform: some rows are valid
-            fail = fail || !mbar_wait(s_full, k & 1u, abort_v, kTimeoutNs);
-            fail = __any_sync(0xffffffffu, fail);
-            // This warp's scores: keys 64 half .. 64 half + 64.
+            fail = fail || !mbar_wait_warp(s_full + g, (uint32_t)(k >> 1) & 1u, abort_v, lim);
+            if (fail) break;
+            tc_fence_after();
+            // Row max over the window's keys.
             float mx = -INFINITY;
-            const int kbase = half * 64;
-            if (!fail) {
-                tc_fence_after();
-                if (active) {
+            if (active) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const int key0 = kbase + c * 32;
-                        if (key0 < len) {  // uniform: the block shares `len`
-                            float v[32];
-                            tmem_ld32(trow + key0, v);
-                            tc_wait_ld();
-                            if (key0 + 32 <= len) {
+                for (int c = 0; c < 4; ++c) {
+                    const int key0 = c * 32;
+                    if (key0 < len) {  // uniform: the block shares `len`
+                        float v[32];
+                        tmem_ld32(t_s + key0, v);
+                        tc_wait_ld();
+                        if (key0 + 32 <= len) {
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
-                            } else {  // the chunk holding the window's end
+                            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
+                        } else {  // the chunk holding the window's end
 #pragma unroll
-                                for (int j = 0; j < 32; ++j)
-                                    if (key0 + j < len) mx = fmaxf(mx, v[j]);
-                            }
+                            for (int j = 0; j < 32; ++j)
+                                if (key0 + j < len) mx = fmaxf(mx, v[j]);
                         }
                     }
                 }
-                red_max[half * kTile + row] = mx;
             }
-            if (quad_sync_any(quad, fail)) {
-                fail = true;
-                break;
-            }
-            mx = fmaxf(red_max[row], red_max[kTile + row]);
             // P = exp2(s * scale - max * scale); zero past the window's end.
             const float neg = -mx * scale_log2e;
             float sum = 0.f;
             if (active) {
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int key0 = kbase + c * 32;
+                for (int c = 0; c < 4; ++c) {
+                    const int key0 = c * 32;
                     if (key0 < len) {
                         const bool whole = key0 + 32 <= len;
-                        float v[1][32];
-                        tmem_ld32(trow + key0, v[0]);
+                        float v[32];
+                        tmem_ld32(t_s + key0, v);
                         tc_wait_ld();
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {  // 8 keys = one 16-byte chunk of P
@@ -359,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int j = q * 8 + 2 * e;
-                                float p0 = ex2_approx(fmaf(v[0][j], scale_log2e, neg));
-                                float p1 = ex2_approx(fmaf(v[0][j + 1], scale_log2e, neg));
+                                float p0 = ex2_approx(fmaf(v[j], scale_log2e, neg));
+                                float p1 = ex2_approx(fmaf(v[j + 1], scale_log2e, neg));
                                 if (!whole) {
                                     p0 = key0 + j < len ? p0 : 0.f;
                                     p1 = key0 + j + 1 < len ? p1 : 0.f;
@@ -375,14 +336,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
                     }
                 }
             }
-            red_sum[half * kTile + row] = sum;
+            const float inv = 1.f / sum;
             // V rows the MMA reads, to fp16 in place (same positions, so the
             // swizzled layout is kept).  Reading V directly needs the TMA
             // barrier's phase observed by this thread (it completed long ago).
-            fail = !v_f16 && !mbar_wait(full + s, use & 1u, abort_v, kTimeoutNs);
-            if (!fail && !v_f16) {
+            if (!v_f16) {
+                fail = !mbar_wait_warp(full + s, (uint32_t)(k / kStages) & 1u, abort_v, lim);
+                if (fail) break;
                 uint4 *vv = reinterpret_cast<uint4 *>(st + 2 * kTileBytes);
-                for (int i = ctid; i < n16 * 128; i += 32 * kComputeWarps) {
+                for (int i = gtid; i < n16 * 128; i += 128) {
                     uint4 u = vv[i];
                     uint32_t *e = reinterpret_cast<uint32_t *>(&u);
 #pragma unroll
@@ -396,20 +358,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
             }
             fence_proxy_async_smem();  // P and V (generic-proxy writes) visible to the MMA
             tc_fence_before();         // S reads done before the next S overwrites it
-            if (quad_sync_any(quad, fail)) {
-                fail = true;
-                break;
-            }
-            const float inv = 1.f / (red_sum[row] + red_sum[kTile + row]);
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
-            // Tile k - 1's output, while O of tile k and S of tile k + 1 compute.
-            if (prev_t >= 0) epilogue(k - 1, prev_t, prev_inv);
-            prev_t = t;
+            if (lane == 0) mbar_arrive(p_full + g);
+            // The group's previous tile's output, while O of this tile and S of
+            // the group's next tile compute.
+            if (prev_k >= 0) epilogue(prev_k, prev_inv);
+            prev_k = k;
             prev_inv = inv;
         }
-        if (!fail && prev_t >= 0) epilogue(k - 1, prev_t, prev_inv);
-        if (fail) signal_abort(status, abort_v);
+        if (!fail && prev_k >= 0) epilogue(prev_k, prev_inv);
+        if (fail && lane == 0) signal_abort(status, abort_v);
     }
     tc_fence_before();
     __syncthreads();
@@ -423,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) window_attn_tc_kernel(
 
 cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                        int d, int heads, int T, int *status, cudaStream_t st,
-                                       bool v_f16) {
+                                       bool v_f16, unsigned long long timeout_ns, int fault_inject) {
     if (n_windows <= 0) return cudaSuccess;
     if (d / heads != kHd || T <= 0) return cudaErrorInvalidValue;
     const cudaError_t e = smem_attr_once<window_attn_tc_kernel>(kSmem);
@@ -435,10 +393,11 @@ cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu
     if (!make_tensor_map_bf16_sw128(&tm, 2, qkv, dims, strides, box)) return cudaErrorInvalidValue;
     const float scale_log2e = 1.4426950408889634f / 8.0f;  // log2(e) / sqrt(64)
     const long tiles = (long)n_windows * heads;
-    const int grid = (int)std::min<long>(tiles, (long)kCtasPerSm * sm_count_cached());
+    const int grid = (int)std::min<long>(tiles, (long)sm_count_cached());
     return launch_pdl(window_attn_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, 1, tm,
                       static_cast<__half *>(out), cu_dev, n_windows, heads, d, scale_log2e, status,
-                      v_f16 ? 1 : 0);
+                      v_f16 ? 1 : 0, timeout_ns ? timeout_ns : 4000ull * 1000ull * 1000ull,
+                      fault_inject);
 }
 
 }  // namespace aut

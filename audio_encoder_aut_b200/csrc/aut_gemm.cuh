@@ -174,11 +174,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *tempty = tfull + 2;
     uint64_t *mma_done = tempty + 2;
     uint64_t *xbar = mma_done + 1;  // [8] per epilogue warp: residual piece landed
-    // [STAGES] odd CTA of a pair: the even CTA has armed the stage's `full`
-    // barrier for the phase the odd CTA is about to load into.
-    uint64_t *armed = xbar + kEpilogueWarps;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(armed + STAGES);
+    // Even CTA of a pair: the odd CTA has reported how many phases of every
+    // stage it loaded (odd_cnt) before exiting its producer loop.
+    uint64_t *exit_bar = xbar + kEpilogueWarps;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(exit_bar + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    uint32_t *odd_cnt = reinterpret_cast<uint32_t *>(abort_flag + 1);  // [STAGES]
+    int *mma_exit = reinterpret_cast<int *>(odd_cnt + STAGES);  // the MMA issuer left its loop
 
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -195,8 +197,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(mma_done, 1);
         for (int w = 0; w < kEpilogueWarps; ++w) mbar_init(xbar + w, 1);
-        for (int st = 0; st < STAGES; ++st) mbar_init(armed + st, 1);
+        mbar_init(exit_bar, 1);
         *abort_flag = 0;
+        *mma_exit = 0;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -230,17 +233,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // ------------------------------------------------ TMA producer --
             // Both CTAs of a pair load their own A rows and B half; the loads of
             // both complete on the even CTA's `full` barrier, which the even CTA
-            // arms with the pair's byte count and then reports armed to the odd
-            // CTA.  The odd CTA loads into a phase only once it is armed, so
-            // every copy either CTA has in flight is counted on a phase the even
-            // CTA waits for before the pair may exit.
+            // arms with the pair's byte count.
             const uint32_t a_bytes =
                 args.conv ? 128u * args.conv_rows * args.conv_cols : (uint32_t)Cfg::A_BYTES;
+            const uint32_t cta_bytes = a_bytes + Cfg::B_BYTES;  // one CTA's loads per stage
             auto arm = [&](int stage) {
-                if (rank == 0) {
-                    mbar_arrive_expect_tx(full + stage, CG * (a_bytes + Cfg::B_BYTES));
-                    if constexpr (CG == 2) mbar_arrive_cluster(map_to_rank(armed + stage, 1));
-                }
+                if (rank == 0) mbar_arrive_expect_tx(full + stage, CG * cta_bytes);
             };
             // Weights (B): k-block kb of the tile whose B rows start at b_row.
             auto load_b = [&](int stage, int kb, int b_row) {
@@ -288,7 +286,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             };
             pdl_wait();  // the previous kernel's outputs (this GEMM's A) are complete
             int stage = 0;
-            uint32_t phase = 0, issued = 0, parity = 0;
+            uint32_t phase = 0;
+            uint32_t cnt[STAGES];  // phases of each stage this CTA has loaded
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s) cnt[s] = 0;
             bool ok = true, skip = args.fault_inject != 0 && blockIdx.x == 0;
             for (int tile = group; ok && tile < total_tiles; tile += n_groups) {
                 const int n_blk = tile % args.num_n_tiles, m_blk = tile / args.num_n_tiles;
@@ -299,18 +300,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ok = false;
                         break;
                     }
-                    if (rank == 1 && !mbar_wait(armed + stage, phase, abort_v, lim)) {
-                        ok = false;
-                        break;
-                    }
                     if (skip) {
                         skip = false;  // injected fault: this stage is never filled
                     } else {
                         arm(stage);
                         load_b(stage, kb, b_row);
                         load_a(stage, kb, m_slot);
-                        issued |= 1u << stage;
-                        parity = (parity & ~(1u << stage)) | (phase << stage);
+#pragma unroll
+                        for (int s = 0; s < STAGES; ++s) cnt[s] += s == stage ? 1u : 0u;
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -319,18 +316,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
             if (!ok) gemm_signal_abort(args, abort_v);
-            if (rank == 0) {
-                // The last load issued on every stage (the odd CTA's included) has
-                // landed before the pair may exit: the odd CTA leaves only through
-                // the cluster barrier at the end, which this CTA reaches after
-                // these waits.  After a failure a phase whose odd half was never
-                // issued does not complete; one shared time limit bounds them all.
-                const uint64_t t0 = global_timer_ns();
-                for (int s = 0; s < STAGES; ++s) {
-                    const uint64_t used = global_timer_ns() - t0;
-                    if ((issued >> s & 1u) && used < lim)
-                        mbar_wait(full + s, parity >> s & 1u, nullptr, lim - used);
+            // Before the block may exit, the last phase loaded into every stage
+            // has landed.  A pair's loads all count on the even CTA's barriers,
+            // and the odd CTA leaves only through the cluster barrier at the end,
+            // which the even CTA reaches after these waits.  After a failure the
+            // two producers may have stopped one phase apart on a stage: the odd
+            // CTA reports its counts, and the even CTA completes the odd half of
+            // a phase the odd CTA never loaded, or arms a phase only the odd CTA
+            // loaded.  One shared time limit bounds all the waits.
+            const uint64_t t0 = global_timer_ns();
+            auto left = [&]() -> uint64_t {
+                const uint64_t used = global_timer_ns() - t0;
+                return used < lim ? lim - used : 0;
+            };
+            if constexpr (CG == 2) {
+                if (rank == 1) {
+#pragma unroll
+                    for (int s = 0; s < STAGES; ++s)
+                        st_shared_cluster_u32(map_to_rank(odd_cnt + s, 0), cnt[s]);
+                    mbar_arrive_cluster(map_to_rank(exit_bar, 0));
+                } else {
+                    // Settle phases only once the MMA issuer has stopped consuming
+                    // them, so that a phase completed here is never read as data.
+                    volatile int *mx = mma_exit;
+                    while (!*mx && left() > 0) {
+                    }
+                    const bool got = mbar_wait_cluster(exit_bar, 0, left());
+#pragma unroll
+                    for (int s = 0; s < STAGES; ++s) {
+                        const uint32_t ce = cnt[s], co = got ? odd_cnt[s] : cnt[s];
+                        if (ce > 0 && co + 1 == ce) mbar_complete_tx(full + s, cta_bytes);
+                        if (ce > 0 && left() > 0) mbar_wait(full + s, (ce - 1) & 1u, nullptr, left());
+                        if (co == ce + 1) {
+                            mbar_arrive_expect_tx(full + s, cta_bytes);
+                            if (left() > 0) mbar_wait(full + s, ce & 1u, nullptr, left());
+                        }
+                    }
                 }
+            } else {
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s)
+                    if (cnt[s] > 0 && left() > 0) mbar_wait(full + s, (cnt[s] - 1) & 1u, nullptr, left());
             }
         }
     } else if (warp == 1) {
@@ -339,21 +365,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t idesc =
                 args.f16 ? idesc_f16_f32(128 * CG, BN) : idesc_bf16_f32(128 * CG, BN);
             constexpr uint16_t kPair = 0x3;
-            // Residual preloaded into the accumulator the MMAs add onto on the
-            // per-row store path; with the TMA-store drain the MMAs start from
-            // zero and the drain adds the residual.
-            const bool resid_mode = args.epi == kEpiResidF32 && !args.tma_out;
             int stage = 0, it = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = group; ok && tile < total_tiles; tile += n_groups, ++it) {
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
-                // Residual mode: wait for the accumulator's preload (phase = use
-                // index); otherwise for the epilogue to have drained it (the phase
-                // before the first use counts as complete).
-                const uint32_t want = resid_mode ? acc_phase : (acc_phase ^ 1u);
-                if (!mbar_wait(tempty + acc, want, abort_v, lim)) {
+                // Wait for the epilogue to have drained the accumulator (the
+                // phase before the first use counts as complete).
+                if (!mbar_wait(tempty + acc, acc_phase ^ 1u, abort_v, lim)) {
                     ok = false;
                     break;
                 }
@@ -378,7 +398,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {  // K = 16 per MMA: +32 bytes in the row
                         if (kk >= ksteps) break;
-                        const uint32_t accumulate = resid_mode || (kb | kk) != 0;
+                        const uint32_t accumulate = (kb | kk) != 0;
                         if constexpr (CG == 2)
                             tc_mma_bf16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
                                              accumulate);
@@ -402,6 +422,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tc_commit(tfull + acc);
             }
             if (!ok) gemm_signal_abort(args, abort_v);
+            *reinterpret_cast<volatile int *>(mma_exit) = 1;
             // Every MMA this thread issued has completed before TMEM is released.
             if constexpr (CG == 2)
                 tc_commit_pair(mma_done, 0x1);
@@ -411,11 +432,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ------------------------------------------------------- epilogue --
-        // Eight warps: TMEM lane quadrant (warp % 4) x column parity (alternate
-        // 16-column chunks); two chunks per TMEM wait.
-        // Residual mode: the accumulator is pre-loaded with x + bias (tcgen05.st)
-        // while the MMAs run on the other accumulator, the MMAs add onto it, and
-        // draining is a plain store - no load sits on the tile's critical path.
+        // Eight warps: TMEM lane quadrant (warp % 4) x column half.  A residual
+        // add is acc + (x + bias) on every path, so that a row's result does not
+        // depend on the tile shape its launch happens to use.
         pdl_wait();  // the residual and the output buffers belong to the previous kernel
         const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
         const int half = (warp - 2) >> 2;
@@ -496,7 +515,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
         };
-        // Residual mode: accumulator `acc` <- x + bias over this thread's row and chunks.
+        // Single-tile residual GEMMs: accumulator `acc` <- x + bias over this
+        // thread's row and the columns this warp drains.
         auto preload = [&](int tile, int acc, bool rel) {
             __syncwarp();  // TMEM stores are warp-wide
             bool valid;
@@ -661,12 +681,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         };
 
-        if (resid_once) {
-            if (group < total_tiles) preload(group, 1, false);
-        } else if (resid && !args.tma_out) {  // the first two accumulators start from the residual
-            int t = group;
-            for (int a = 0; a < 2 && t < total_tiles; ++a, t += n_groups) preload(t, a, true);
-        }
+        if (resid_once && group < total_tiles) preload(group, 1, false);
         int it = 0;
         for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
             const int acc = it & 1;
@@ -744,7 +759,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             store_bf16x16(o + args.N, lo);
                             break;
                         }
-                        case kEpiResidF32:  // accumulator already holds x + bias + X W^T
+                        case kEpiResidF32: {  // acc + (x + bias), x read back from the output
+                            float r[16];
+                            const float4 *xp = reinterpret_cast<const float4 *>(rp + n0);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 e = xp[q];
+                                r[4 * q] = e.x;
+                                r[4 * q + 1] = e.y;
+                                r[4 * q + 2] = e.z;
+                                r[4 * q + 3] = e.w;
+                            }
+                            add_bias16(r, args.bias, n0);
+                            float4 *p = reinterpret_cast<float4 *>(rp + n0);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                p[q] = make_float4(v[4 * q] + r[4 * q], v[4 * q + 1] + r[4 * q + 1],
+                                                   v[4 * q + 2] + r[4 * q + 2], v[4 * q + 3] + r[4 * q + 3]);
+                            break;
+                        }
                         case kEpiF32:
                         case kEpiPackTokens: {
                             if (args.epi == kEpiPackTokens && args.pos) {
@@ -771,15 +804,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
             }
-            if (resid && !args.tma_out) {
-                const int next = tile + 2 * n_groups;  // the tile this accumulator serves next
-                if (next < total_tiles) {
-                    tc_fence_before();  // finish reading the drained values before rewriting
-                    preload(next, acc, true);
-                }
-            } else {
-                release(acc);
-            }
+            release(acc);
         }
         if (!ok && lane == 0) gemm_signal_abort(args, abort_v);
         // The staged stores have read shared memory before the block may exit;

@@ -92,13 +92,17 @@ cudaError_t launch_to_f16(const void *src, void *dst, size_t n, cudaStream_t st)
 // the head_dim-64 tensor-core path (T > 0) accepts it.
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                     int d, int heads, cudaStream_t st, int T = -1,
-                                    int *status = nullptr, bool v_f16 = false);
+                                    int *status = nullptr, bool v_f16 = false,
+                                    unsigned long long timeout_ns = 0, int fault_inject = 0);
 // Whether launch_window_attention takes the tensor-core path.
 inline bool window_attention_uses_tc(int d, int heads, int T) { return d / heads == 64 && T > 0; }
 // tcgen05 variant for head_dim 64 (aut_attention.cu); T = rows of qkv.
+// timeout_ns bounds every pipeline wait (0: 4 s); fault_inject leaves the first
+// block's first stage unfilled (tests of the time-out path only).
 cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                        int d, int heads, int T, int *status, cudaStream_t st,
-                                       bool v_f16 = false);
+                                       bool v_f16 = false, unsigned long long timeout_ns = 0,
+                                       int fault_inject = 0);
 // bf16 tensor map with 128-byte swizzle (aut_gemm.cu): dims innermost first,
 // strides in bytes for dims 1.., box in elements.
 bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,

@@ -77,6 +77,32 @@ AUT_DEV bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
     return __all_sync(0xffffffffu, ok);
 }
 
+// Completes `bytes` of the current phase's expected transaction count without
+// a copy (for bytes that will never arrive).
+AUT_DEV void mbar_complete_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// mbar_wait with acquire at cluster scope: data another CTA of the cluster
+// stored before its release-arrive on `bar` is visible once this returns true.
+AUT_DEV bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+}
+
 // -------------------------------------------------------------------- TMA --
 AUT_DEV void tma_prefetch_desc(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -355,6 +381,9 @@ AUT_DEV uint32_t map_to_rank(const void *p, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
     return r;
+}
+AUT_DEV void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 AUT_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)

@@ -241,6 +241,18 @@ aut_status aut_window_attention(const void *qkv, void *out, int32_t T, int32_t d
                                 const int32_t *cu_seqlens, int32_t num_windows,
                                 void *workspace, size_t ws_bytes, aut_stream_t stream);
 
+/* aut_window_attention with control over its failure path, for tests:
+ * timeout_ms bounds every pipeline wait of the head_dim-64 tensor-core kernel
+ * (0 = default of 4000 ms); flags AUT_ATTN_FAULT_INJECT leaves the first
+ * block's first operand stage unfilled, so that its consumers' waits run out,
+ * the kernel writes AUT_ERR_TIMEOUT to the workspace's status word and returns
+ * (head_dim 64 only; AUT_ERR_UNSUPPORTED otherwise); 0 for normal use. */
+#define AUT_ATTN_FAULT_INJECT 1
+aut_status aut_window_attention_ex(const void *qkv, void *out, int32_t T, int32_t d,
+                                   int32_t heads, const int32_t *cu_seqlens, int32_t num_windows,
+                                   void *workspace, size_t ws_bytes, int32_t timeout_ms,
+                                   int32_t flags, aut_stream_t stream);
+
 /* Window attention that allocates nothing, for callers that cannot allocate
  * device memory: code whose device memory belongs to another allocator that
  * forbids raw cudaMalloc, or code running where allocation is not allowed

@@ -200,3 +200,34 @@ def test_pipeline_wait_timeout_returns_status_and_gpu_stays_usable(mode):
     assert st == A.AUT_OK and A.aut_check_status_word(status.data_ptr()) == A.AUT_OK
     ref = x.float().cpu().numpy().astype(np.float64) @ w.float().cpu().numpy().astype(np.float64).T
     assert_rows_close(y.float().cpu().numpy(), ref, "linear after timeout")
+
+
+def test_attention_wait_timeout_returns_status_and_gpu_stays_usable():
+    """The tensor-core attention with its first block's first operand stage
+    never filled: the MMA's bounded wait runs out, the softmax groups and the
+    producer leave on the abort flag, the kernel writes AUT_ERR_TIMEOUT to the
+    workspace's status word and returns; the next launch on the same context
+    computes the right result."""
+    heads, hd, lens = 20, 64, [104, 104, 50, 77]
+    d = heads * hd
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    T = cu[-1]
+    qkv = _rand((T, 3 * d), 13, 1.0)
+    qd = _dev(qkv, torch.bfloat16)
+    out = torch.empty((T, d), dtype=torch.float16, device="cuda")
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    st = A.aut_window_attention_ex(qd.data_ptr(), out.data_ptr(), T, d, heads, cu, ws.data_ptr(),
+                                   ws.numel(), 200, A.ATTN_FAULT_INJECT, _stream())
+    assert st == A.AUT_OK
+    torch.cuda.synchronize()
+    assert A.aut_check(ws.data_ptr()) == A.AUT_ERR_TIMEOUT
+    st = A.aut_window_attention_ex(qd.data_ptr(), out.data_ptr(), T, d, heads, cu, ws.data_ptr(),
+                                   ws.numel(), 0, 0, _stream())
+    torch.cuda.synchronize()
+    assert st == A.AUT_OK and A.aut_check(ws.data_ptr()) == A.AUT_OK
+    ref = O.window_attention(qkv.astype(np.float64), cu, heads)
+    vmax = np.abs(qkv[:, 2 * d:]).max()
+    assert_f16_output_close(out.float().cpu().numpy().astype(np.float64), ref,
+                            "attention after timeout", atol=2e-4 * vmax)
