@@ -169,7 +169,8 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
     void *planes2 = c.at<void>(c.L.planes2);
     void *y3 = c.at<void>(c.L.y3);
     const int p1_rows = G * kP1Rows, p2_rows = G * kP2Rows;
-    AUT_TRY(cuda_status(launch_zero_plane_pads(planes2, p2_rows, G, C, c.st)));
+    AUT_TRY(cuda_status(
+        launch_zero_plane_pads(planes2, p2_rows, G, kP2Rows, kP2Cols, true, C, c.st)));
     AUT_TRY(c.mark(AUT_K_ZERO_PADS));
     for (int c0 = 0; c0 < n_ch; c0 += G) {
         const int g = std::min(G, n_ch - c0);

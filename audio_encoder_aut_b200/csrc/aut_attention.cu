@@ -60,7 +60,9 @@ constexpr int kTileBytes = kTile * kHd * 2;  // 16 KiB
 constexpr int kStages = 4;
 constexpr int kStageBytes = 3 * kTileBytes;  // Q | K | V; P (fp16, 128 x 128) overwrites Q | K
 constexpr int kGroups = 2;                   // softmax groups (four warps each)
-constexpr int kOffBar = kStages * kStageBytes;
+constexpr int kOffWin = kStages * kStageBytes;
+constexpr int kWinCache = 512;  // (row0, length) of a CTA's first local tiles' windows
+constexpr int kOffBar = kOffWin + kWinCache * 8;
 // full[kStages], empty[kStages], s_full[2], p_full[2], o_full[4], o_empty[4], mma_done
 constexpr int kNumBars = 2 * kStages + 2 * kGroups + 4 + 4 + 1;
 constexpr int kSmem = 1024 + kOffBar + kNumBars * 8 + 16;
@@ -92,6 +94,19 @@ __device__ __forceinline__ void window_of(const int *cu, int w, int *s0, int *le
     *len = cu[w + 1] - *s0;
     *n16 = max(1, (*len + 15) >> 4);
 }
+// The same from the CTA's shared-memory cache of its local tiles' windows
+// (entries past the cache are read from cu_seqlens).
+__device__ __forceinline__ void local_window(const int2 *cache, const int *cu, int k, int w, int *s0,
+                                             int *len, int *n16) {
+    if (k < kWinCache) {
+        const int2 e = cache[k];
+        *s0 = e.x;
+        *len = e.y;
+        *n16 = max(1, (e.y + 15) >> 4);
+    } else {
+        window_of(cu, w, s0, len, n16);
+    }
+}
 
 __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_qkv, __half *__restrict__ out, const int *__restrict__ cu,
@@ -100,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    int2 *wcache = reinterpret_cast<int2 *>(sm + kOffWin);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + kOffBar);
     uint64_t *empty = full + kStages;
     uint64_t *s_full = empty + kStages;  // [2] S of the group's tile in TMEM
@@ -144,6 +160,14 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
     // This CTA's tiles: blockIdx.x + k gridDim.x for k < n_local.
     const int n_local = blockIdx.x < n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     auto tile_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
+    // Every role needs each tile's window: read them from cu_seqlens once, in
+    // parallel, instead of one dependent global load per tile and role.
+    for (int k = threadIdx.x; k < min(n_local, kWinCache); k += kThreads) {
+        const int w = tile_of(k) / heads;
+        const int a = cu[w];
+        wcache[k] = make_int2(a, cu[w + 1] - a);
+    }
+    __syncthreads();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -160,7 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
                 }
                 if (fault_inject && blockIdx.x == 0 && k == 0) continue;  // never filled
                 uint8_t *st = sm + s * kStageBytes;
-                const int s0 = cu[w];
+                int s0, len, n16;
+                local_window(wcache, cu, k, w, &s0, &len, &n16);
                 mbar_arrive_expect_tx(full + s, kStageBytes);
                 tma_load_2d(st, &tm_qkv, full + s, h * kHd, s0);
                 tma_load_2d(st + kTileBytes, &tm_qkv, full + s, d + h * kHd, s0);
@@ -186,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
             // S of local tile k into its group's S buffer.
             auto issue_s = [&](int k) -> bool {
                 int s0, len, n16;
-                window_of(cu, tile_of(k) / heads, &s0, &len, &n16);
+                local_window(wcache, cu, k, tile_of(k) / heads, &s0, &len, &n16);
                 const int s = k % kStages;
                 if (!mbar_wait(full + s, (uint32_t)(k / kStages) & 1u, abort_v, lim)) return false;
                 tc_fence_after();
@@ -202,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
             for (int k = 0; ok && k < n_local && k < kGroups; ++k) ok = issue_s(k);
             for (int k = 0; ok && k < n_local; ++k) {
                 int s0, len, n16;
-                window_of(cu, tile_of(k) / heads, &s0, &len, &n16);
+                local_window(wcache, cu, k, tile_of(k) / heads, &s0, &len, &n16);
                 const int g = k & 1, ob = 2 * g + ((k >> 1) & 1);
                 uint8_t *st = sm + (k % kStages) * kStageBytes;
                 // P of tile k is in shared memory (and S has been read); the O
@@ -241,63 +266,71 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
         auto epilogue = [&](int kk, float inv) {
             const int t = tile_of(kk), w = t / heads, h = t - w * heads;
             int s0, len, n16;
-            window_of(cu, w, &s0, &len, &n16);
+            local_window(wcache, cu, kk, w, &s0, &len, &n16);
             const int ob = 2 * g + ((kk >> 1) & 1);
             fail = fail || !mbar_wait_warp(o_full + ob, (uint32_t)(kk >> 2) & 1u, abort_v, lim);
             if (fail) return;
             tc_fence_after();
             const bool active = quad * 32 < len;
-            float o[2][32];
+            __half *dst = out + (size_t)(s0 + row) * d + h * kHd;
             if (active) {
-                tmem_ld32(trow + kColO + ob * kHd, o[0]);
-                tmem_ld32(trow + kColO + ob * kHd + 32, o[1]);
-                tc_wait_ld();
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {  // 32 output columns per TMEM load
+                    float o[32];
+                    tmem_ld32(trow + kColO + ob * kHd + 32 * hh, o);
+                    tc_wait_ld();
+                    if (row < len) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                pk[e] = pack_f16x2_sat(o[q * 8 + 2 * e] * inv, o[q * 8 + 2 * e + 1] * inv);
+                            *reinterpret_cast<uint4 *>(dst + 32 * hh + q * 8) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(o_empty + ob);
-            if (active && row < len) {
-                __half *dst = out + (size_t)(s0 + row) * d + h * kHd;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        pk[e] = pack_f16x2_sat(o[q >> 2][(q & 3) * 8 + 2 * e] * inv,
-                                               o[q >> 2][(q & 3) * 8 + 2 * e + 1] * inv);
-                    *reinterpret_cast<uint4 *>(dst + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
         };
         int prev_k = -1;
         float prev_inv = 0.f;
         for (int k = g; k < n_local; k += kGroups) {
             int s0, len, n16;
-            window_of(cu, tile_of(k) / heads, &s0, &len, &n16);
+            local_window(wcache, cu, k, tile_of(k) / heads, &s0, &len, &n16);
             const int s = k % kStages;
             uint8_t *st = sm + s * kStageBytes;
             const uint32_t t_s = trow + g * kTile;
             const bool active = quad * 32 < len;  // warp-uniform: some rows are valid
+            const int nch = (len + 31) >> 5;      // 32-key chunks holding the window's keys
             fail = fail || !mbar_wait_warp(s_full + g, (uint32_t)(k >> 1) & 1u, abort_v, lim);
             if (fail) break;
             tc_fence_after();
-            // Row max over the window's keys.
+            // Row max over the window's keys: the scores come out of TMEM 64 keys
+            // (two 32-key chunks) per wait.
             float mx = -INFINITY;
             if (active) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int key0 = c * 32;
-                    if (key0 < len) {  // uniform: the block shares `len`
-                        float v[32];
-                        tmem_ld32(t_s + key0, v);
+                for (int c0 = 0; c0 < 4; c0 += 2) {
+                    if (c0 < nch) {
+                        float v[2][32];
+                        tmem_ld32(t_s + c0 * 32, v[0]);
+                        if (c0 + 1 < nch) tmem_ld32(t_s + c0 * 32 + 32, v[1]);
                         tc_wait_ld();
-                        if (key0 + 32 <= len) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
-                        } else {  // the chunk holding the window's end
+                        for (int u = 0; u < 2; ++u) {
+                            const int key0 = (c0 + u) * 32;
+                            if (key0 + 32 <= len) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (key0 + j < len) mx = fmaxf(mx, v[j]);
+                                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[u][j]);
+                            } else if (key0 < len) {  // the chunk holding the window's end
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (key0 + j < len) mx = fmaxf(mx, v[u][j]);
+                            }
                         }
                     }
                 }
@@ -307,31 +340,37 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
             float sum = 0.f;
             if (active) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int key0 = c * 32;
-                    if (key0 < len) {
-                        const bool whole = key0 + 32 <= len;
-                        float v[32];
-                        tmem_ld32(t_s + key0, v);
+                for (int c0 = 0; c0 < 4; c0 += 2) {
+                    if (c0 < nch) {
+                        float v[2][32];
+                        tmem_ld32(t_s + c0 * 32, v[0]);
+                        if (c0 + 1 < nch) tmem_ld32(t_s + c0 * 32 + 32, v[1]);
                         tc_wait_ld();
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {  // 8 keys = one 16-byte chunk of P
-                            uint32_t ph[4];
+                        for (int u = 0; u < 2; ++u) {
+                            const int key0 = (c0 + u) * 32;
+                            if (key0 < len) {
+                                const bool whole = key0 + 32 <= len;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = q * 8 + 2 * e;
-                                float p0 = ex2_approx(fmaf(v[j], scale_log2e, neg));
-                                float p1 = ex2_approx(fmaf(v[j + 1], scale_log2e, neg));
-                                if (!whole) {
-                                    p0 = key0 + j < len ? p0 : 0.f;
-                                    p1 = key0 + j + 1 < len ? p1 : 0.f;
+                                for (int q = 0; q < 4; ++q) {  // 8 keys = one 16-byte chunk of P
+                                    uint32_t ph[4];
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const int j = q * 8 + 2 * e;
+                                        float p0 = ex2_approx(fmaf(v[u][j], scale_log2e, neg));
+                                        float p1 = ex2_approx(fmaf(v[u][j + 1], scale_log2e, neg));
+                                        if (!whole) {
+                                            p0 = key0 + j < len ? p0 : 0.f;
+                                            p1 = key0 + j + 1 < len ? p1 : 0.f;
+                                        }
+                                        sum += p0 + p1;
+                                        __half2 hp = __floats2half2_rn(p0, p1);
+                                        ph[e] = *reinterpret_cast<uint32_t *>(&hp);
+                                    }
+                                    *reinterpret_cast<uint4 *>(st + p_chunk_offset(row, key0 / 8 + q)) =
+                                        make_uint4(ph[0], ph[1], ph[2], ph[3]);
                                 }
-                                sum += p0 + p1;
-                                __half2 hp = __floats2half2_rn(p0, p1);
-                                ph[e] = *reinterpret_cast<uint32_t *>(&hp);
                             }
-                            *reinterpret_cast<uint4 *>(st + p_chunk_offset(row, key0 / 8 + q)) =
-                                make_uint4(ph[0], ph[1], ph[2], ph[3]);
                         }
                     }
                 }

@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // CTA reports its counts, and the even CTA completes the odd half of
             // a phase the odd CTA never loaded, or arms a phase only the odd CTA
             // loaded.  One shared time limit bounds all the waits.
-            const uint64_t t0 = global_timer_ns();
+            uint64_t t0 = global_timer_ns();
             auto left = [&]() -> uint64_t {
                 const uint64_t used = global_timer_ns() - t0;
                 return used < lim ? lim - used : 0;
@@ -338,9 +338,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 } else {
                     // Settle phases only once the MMA issuer has stopped consuming
                     // them, so that a phase completed here is never read as data.
+                    // The issuer leaves its loop within one wait limit of a
+                    // failure; the bound here is well past that, so this spin
+                    // cannot run out first and settle a phase it still waits on.
                     volatile int *mx = mma_exit;
-                    while (!*mx && left() > 0) {
+                    while (!*mx && global_timer_ns() - t0 < 4 * lim) {
                     }
+                    t0 = global_timer_ns();
                     const bool got = mbar_wait_cluster(exit_bar, 0, left());
 #pragma unroll
                     for (int s = 0; s < STAGES; ++s) {

@@ -111,31 +111,35 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
         }
 }
 
-// Zero row, zero column and (odd-column planes) the missing last column of
-// conv3's input planes: the conv2 epilogue never writes them.
-__global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int plane_rows, int C) {
+// Zero row and zero column of every chunk's rows of the four phase planes, and
+// (odd-column planes with `last_col`) their last column: the kernels that fill
+// the planes never write them.  Planes [4][plane_rows][cols][C], chunk_rows
+// rows per chunk, row 0 of a chunk and column 0 the zero borders.
+__global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int plane_rows,
+                                                              int chunk_rows, int cols,
+                                                              int last_col, int C) {
     pdl_trigger();
     pdl_wait();
     const int cl = blockIdx.x, plane = blockIdx.y;
     const int CP = C >> 1;
-    const size_t row0 = (size_t)plane * plane_rows + (size_t)cl * kP2Rows;
-    const int extra = (plane & 1) ? (kP2Rows - 1) : 0;  // column kP2Cols - 1 of rows 1..16
-    const int n = (kP2Cols + (kP2Rows - 1) + extra) * CP;
+    const size_t row0 = (size_t)plane * plane_rows + (size_t)cl * chunk_rows;
+    const int extra = (last_col && (plane & 1)) ? (chunk_rows - 1) : 0;
+    const int n = (cols + (chunk_rows - 1) + extra) * CP;
     for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
         const int e = idx / CP, cp = idx - e * CP;
         size_t row;
         int col;
-        if (e < kP2Cols) {
+        if (e < cols) {
             row = row0;
             col = e;
-        } else if (e < kP2Cols + kP2Rows - 1) {
-            row = row0 + 1 + (e - kP2Cols);
+        } else if (e < cols + chunk_rows - 1) {
+            row = row0 + 1 + (e - cols);
             col = 0;
         } else {
-            row = row0 + 1 + (e - kP2Cols - (kP2Rows - 1));
-            col = kP2Cols - 1;
+            row = row0 + 1 + (e - cols - (chunk_rows - 1));
+            col = cols - 1;
         }
-        reinterpret_cast<uint32_t *>(planes + (row * kP2Cols + col) * C)[cp] = 0u;
+        reinterpret_cast<uint32_t *>(planes + (row * cols + col) * C)[cp] = 0u;
     }
 }
 
@@ -478,11 +482,12 @@ cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int c
                       static_cast<bf16 *>(planes), plane_rows, C);
 }
 
-cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int C,
-                                   cudaStream_t st) {
+cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int chunk_rows,
+                                   int cols, bool last_col, int C, cudaStream_t st) {
     if (n_chunks <= 0) return cudaSuccess;
     return launch_pdl(zero_plane_pads_kernel, dim3(n_chunks, 4), dim3(256), 0, st, 1,
-                      static_cast<bf16 *>(planes), plane_rows, C);
+                      static_cast<bf16 *>(planes), plane_rows, chunk_rows, cols, last_col ? 1 : 0,
+                      C);
 }
 
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,

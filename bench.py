@@ -41,11 +41,15 @@ METRIC = "encoded audio-seconds/s on 1 B200 (bf16); tokens/s and % of bf16 TC pe
 UNIT = "audio-s/s"
 
 
-# DRAM bytes (read + write) per gemm_tc_kernel launch, mean over the 101 GEMM
-# launches of one omni_16req forward, from one ncu capture of this kernel
-# version (dram__bytes_read.sum + dram__bytes_write.sum, cold caches).  None
-# whenever the kernel has changed since that capture.
-GEMM_DRAM_BYTES_PER_LAUNCH = None
+# The roofline's kernel: gemm_tc_kernel over the layer GEMMs (qkv, o_proj, fc1,
+# fc2; 4 launches per layer).  DRAM bytes (read + write) per launch, mean over
+# layer 0's four launches of one omni_16req forward (every layer has the same
+# shapes), from one ncu capture of the current kernel: dram__bytes_read.sum +
+# dram__bytes_write.sum of 18.26 / 28.34 / 21.55 / 63.19 MB (the command and
+# the table are in profiles/gemm_tc_kernel_dram_omni_16req.md).  Set to None
+# whenever the kernel changes.
+LAYER_GEMM_DRAM_BYTES_PER_LAUNCH = 32.835e6
+LAYER_GEMMS = ("qkv", "o_proj", "fc1", "fc2")
 
 
 def peaks():
@@ -63,29 +67,44 @@ def _half(n):
 
 
 def credited_flops(cfg, lens, cu):
-    """Algorithmic FLOPs of one forward, valid positions only: the stem per chunk
-    (conv1, conv2, conv3 on the output positions the chunk's valid frames reach,
-    conv_out on its kept tokens), 2 (4 d^2 + 2 d F) per token and layer for the
-    layer GEMMs, 4 d len^2 per window and layer for attention, 2 (d^2 + d O) per
-    token for the projector.  Returns (total, tcgen05-GEMM part)."""
+    """Algorithmic FLOPs of one forward, valid positions only, by kernel kind:
+    the stem per chunk (conv1, conv2, conv3 on the output positions the chunk's
+    valid frames reach, conv_out on its kept tokens), 2 d (3 d), 2 d d, 2 d F,
+    2 F d per token and layer for qkv, o_proj, fc1, fc2, 4 d len^2 per window
+    and layer for attention, 2 d d and 2 d O per token for the projector."""
     C, d, F, O, L = (cfg.downsample_hidden_size, cfg.d_model, cfg.encoder_ffn_dim,
                      cfg.output_dim, cfg.encoder_layers)
-    conv1 = conv23 = conv_out = 0
+    k = dict.fromkeys(["conv1", "conv2", "conv3", "conv_out"], 0)
     for n in lens:
         for s in range(0, n, 100):
             v = min(100, n - s)
             f1 = _half(v)
             f2 = _half(f1)
             f3 = _half(f2)
-            conv1 += 2 * C * 9 * 64 * f1
-            conv23 += 2 * C * 9 * C * (32 * f2 + 16 * f3)
-            conv_out += 2 * f3 * 16 * C * d
+            k["conv1"] += 2 * C * 9 * 64 * f1
+            k["conv2"] += 2 * C * 9 * C * 32 * f2
+            k["conv3"] += 2 * C * 9 * C * 16 * f3
+            k["conv_out"] += 2 * f3 * 16 * C * d
     T = cu[-1]
-    layers = L * 2 * (4 * d * d + 2 * d * F) * T
-    attn = L * 4 * d * sum((b - a) ** 2 for a, b in zip(cu[:-1], cu[1:]))
-    proj = 2 * (d * d + d * O) * T
-    gemm = conv23 + conv_out + layers + proj
-    return gemm + conv1 + attn, gemm
+    k["qkv"] = L * 2 * T * 3 * d * d
+    k["o_proj"] = L * 2 * T * d * d
+    k["fc1"] = L * 2 * T * d * F
+    k["fc2"] = L * 2 * T * F * d
+    k["attention"] = L * 4 * d * sum((b - a) ** 2 for a, b in zip(cu[:-1], cu[1:]))
+    k["proj1"] = 2 * T * d * d
+    k["proj2"] = 2 * T * d * O
+    return k
+
+
+def layer_gemm_operand_bytes(cfg, T):
+    """Mean bytes a layer GEMM must read once (A, W, and the fp32 residual of
+    o_proj and fc2; outputs stay in L2): the algorithmic traffic per launch."""
+    d, F = cfg.d_model, cfg.encoder_ffn_dim
+    qkv = 2 * T * d + 2 * 3 * d * d
+    o = 2 * T * d + 2 * d * d + 4 * T * d
+    fc1 = 2 * T * d + 2 * F * d
+    fc2 = 2 * T * F + 2 * d * F + 4 * T * d
+    return (qkv + o + fc1 + fc2) / 4
 
 
 # ---------------------------------------------------------------- clocks ----
@@ -294,7 +313,8 @@ def our_arm(args, rank, world, local_rank):
         dist.all_reduce(job_T)
     value = job_audio_s * args.steps / (total_ms / 1e3)
     tokens_s = int(job_T.item()) * args.steps / (total_ms / 1e3)
-    flops, gemm_flops = credited_flops(cfg, lens, cu)
+    kflops = credited_flops(cfg, lens, cu)
+    flops = sum(kflops.values())
     pk, pk_sus, hbm, pk_src = peaks()
 
     # Per-kernel breakdown: the same forward captured as a graph with an event
@@ -329,10 +349,18 @@ def our_arm(args, rank, world, local_rank):
             k = A.KERNEL_KINDS[kinds[i]]
             per_kind.setdefault(k, []).append(events[i].elapsed_time(events[i + 1]))
     kind_ms = {k: sum(v) / n_trace for k, v in per_kind.items()}
-    gemm_launches = sum(len(v) for k, v in per_kind.items() if k in A.GEMM_KINDS) / n_trace
-    gemm_ms = sum(kind_ms[k] for k in kind_ms if k in A.GEMM_KINDS)
+    # The roofline's kernel: the layer GEMMs.  achieved = their credited FLOPs
+    # per launch / their mean launch time (from the event-timed replay).
+    gemm_launches = sum(len(per_kind[k]) for k in LAYER_GEMMS if k in per_kind) / n_trace
+    gemm_ms = sum(kind_ms[k] for k in LAYER_GEMMS if k in kind_ms)
     gemm_avg_ms = gemm_ms / gemm_launches
+    gemm_flops = sum(kflops[k] for k in LAYER_GEMMS)
     achieved = gemm_flops / gemm_launches / (gemm_avg_ms / 1e3) / 1e12
+    per_kind_tflops = {k: {"tflops": round(kflops[k] / (kind_ms[k] / 1e3) / 1e12, 1),
+                           "frac": round(kflops[k] / (kind_ms[k] / 1e3) / 1e12 / pk, 3)}
+                       for k in kflops if k in kind_ms and kind_ms[k] > 0 and k in A.GEMM_KINDS}
+    all_gemm = sum(kflops[k] for k in A.GEMM_KINDS if k in kflops)
+    all_gemm_ms = sum(kind_ms[k] for k in A.GEMM_KINDS if k in kind_ms)
 
     # End to end through the public API: every step copies its features in from
     # pinned host memory and its fp32 result back out; the copies of steps
@@ -383,13 +411,20 @@ def our_arm(args, rank, world, local_rank):
             "pct_bf16_peak_sustained": 100 * flops / (ms / 1e3) / 1e12 / pk_sus,
             "step_ms_p50_p95_p99": [pct(50), pct(95), pct(99)],
             "credited_gflop_per_step": flops / 1e9,
-            "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (all tcgen05 GEMM launches)",
+            "roofline": {"bound": "tensor",
+                         "kernel": "gemm_tc_kernel on the layer GEMMs (qkv, o_proj, fc1, fc2 "
+                                   "x layers)",
                          "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
                          "frac": achieved / pk, "peak_source": f"{pk_src} bf16 burst",
                          "peak_sustained": pk_sus, "launches_per_step": gemm_launches,
-                         "avg_launch_ms": gemm_avg_ms, "traffic": GEMM_DRAM_BYTES_PER_LAUNCH,
+                         "avg_launch_ms": gemm_avg_ms,
+                         "traffic": LAYER_GEMM_DRAM_BYTES_PER_LAUNCH,
                          "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + "
-                                         "dram__bytes_write.sum, mean over one forward's GEMMs)"},
+                                         "dram__bytes_write.sum, mean over layer 0's qkv, "
+                                         "o_proj, fc1, fc2)",
+                         "algorithmic_bytes_per_launch": layer_gemm_operand_bytes(cfg, T),
+                         "per_gemm": per_kind_tflops,
+                         "all_gemms_frac": all_gemm / (all_gemm_ms / 1e3) / 1e12 / pk},
             "kernel_ms_per_step": {k: round(v, 4) for k, v in sorted(kind_ms.items(), key=lambda x: -x[1])},
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": h_feats.numel() * h_feats.element_size(),
@@ -453,7 +488,7 @@ def sweep(args):
             torch.cuda.synchronize()
             ms.append(a.elapsed_time(b))
         t = sorted(ms)[len(ms) // 2]
-        flops = credited_flops(cfg, lens, cu)[0]
+        flops = sum(credited_flops(cfg, lens, cu).values())
         print(json.dumps({"sweep_tokens": T, "requests": len(lens), "audio_seconds": sum(lens) / 100,
                           "ms_per_step": t, "audio_s_per_s": sum(lens) / 100 / (t / 1e3),
                           "tokens_per_s": T / (t / 1e3), "tflops": flops / (t / 1e3) / 1e12,
