@@ -140,19 +140,20 @@ aut_status linear(const Ctx &c, const void *a, const void *w, const void *b, voi
     return c.mark(kind);
 }
 
+// The chunk table and cu_seqlens lie next to each other in the workspace
+// (chunks, padding, cu); one upload writes the whole span.
 aut_status upload_plan(const Ctx &c, const Plan &p) {
-    std::vector<int32_t> words;
-    words.reserve(p.chunks.size() * 4);
+    const size_t cu_word = (c.L.cu - c.L.chunks) / 4;
+    std::vector<int32_t> words(cu_word + p.cu_seqlens.size(), 0);
+    size_t i = 0;
     for (const ChunkInfo &ci : p.chunks) {
-        words.push_back(ci.request);
-        words.push_back(ci.frame0);
-        words.push_back(ci.valid_frames);
-        words.push_back(ci.token0);
+        words[i++] = ci.request;
+        words[i++] = ci.frame0;
+        words[i++] = ci.valid_frames;
+        words[i++] = ci.token0;
     }
+    std::copy(p.cu_seqlens.begin(), p.cu_seqlens.end(), words.begin() + cu_word);
     AUT_TRY(cuda_status(launch_upload(words.data(), words.size(), c.at<int32_t>(c.L.chunks), c.st)));
-    AUT_TRY(c.mark(AUT_K_UPLOAD));
-    AUT_TRY(cuda_status(
-        launch_upload(p.cu_seqlens.data(), p.cu_seqlens.size(), c.at<int32_t>(c.L.cu), c.st)));
     return c.mark(AUT_K_UPLOAD);
 }
 
@@ -169,13 +170,10 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
     void *planes2 = c.at<void>(c.L.planes2);
     void *y3 = c.at<void>(c.L.y3);
     const int p1_rows = G * kP1Rows, p2_rows = G * kP2Rows;
-    AUT_TRY(cuda_status(
-        launch_zero_plane_pads(planes2, p2_rows, G, kP2Rows, kP2Cols, true, C, c.st)));
-    AUT_TRY(c.mark(AUT_K_ZERO_PADS));
     for (int c0 = 0; c0 < n_ch; c0 += G) {
         const int g = std::min(G, n_ch - c0);
         AUT_TRY(cuda_status(launch_conv1(feats, T_max, chunks, c0, g, c.w->conv1_w, c.w->conv1_b,
-                                         planes1, p1_rows, C, c.st)));
+                                         planes1, p1_rows, planes2, p2_rows, C, c.st)));
         AUT_TRY(c.mark(AUT_K_CONV1));
         ConvLaunch k2{};
         k2.planes = planes1;

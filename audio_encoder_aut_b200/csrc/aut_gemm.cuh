@@ -78,21 +78,25 @@ struct GemmCfg {
     static constexpr int B_ROWS = BN / CG;
     static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES_FIT = 196608 / STAGE_BYTES;
+    // Output staging for the TMA-store epilogue: two boxes of 32 rows x 128
+    // bytes per epilogue warp (128-byte-swizzled), used alternately so that one
+    // piece's store drains while the next piece is computed; only for tile
+    // widths whose half is a whole number of 32-column fp32 pieces (no other
+    // width can use it, and shared memory left unallocated serves as L1 cache).
+    static constexpr int STAGING_BYTES = (BN / 2) % 32 == 0 ? kEpilogueWarps * 2 * 4096 : 0;
+    static constexpr int BAR_BYTES = 384;
+    static constexpr int SMEM_LIMIT = 232448;  // dynamic shared memory per block on sm_100
+    static constexpr int STAGES_FIT =
+        (SMEM_LIMIT - 1024 - STAGING_BYTES - BAR_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static constexpr int TMEM_COLS = (2 * BN <= 32)    ? 32
                                      : (2 * BN <= 64)  ? 64
                                      : (2 * BN <= 128) ? 128
                                      : (2 * BN <= 256) ? 256
                                                        : 512;
-    // Output staging for the TMA-store epilogue: 32 rows x 128 bytes per
-    // epilogue warp (one 128-byte-swizzled box), for tile widths whose half is
-    // a whole number of 32-column fp32 pieces (no other width can use it, and
-    // shared memory left unallocated serves as L1 cache).
-    static constexpr int STAGING_BYTES = (BN / 2) % 32 == 0 ? 8 * 4096 : 0;
-    static constexpr int BAR_BYTES = 384;
     static constexpr int SMEM_BYTES =
         1024 /*alignment slack*/ + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
+    static_assert(STAGES >= 3, "at least three operand stages");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
     static_assert(B_ROWS % 8 == 0, "each CTA holds whole 8-row swizzle atoms of B");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay aligned");
@@ -456,11 +460,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool x_pending = false;  // lane 0: a residual load has not been waited for
         // Residual piece (32 rows x 32 fp32) of `tile` at column offset `col`
         // into this warp's staging box; lane 0 only.
-        auto load_x = [&](int tile, int col) {
+        uint8_t *const my_boxes = staging + (warp - 2) * 8192;  // two 4 KB boxes
+        // Stores this warp has issued (warp-uniform); a piece fills box piece & 1,
+        // so the most recent store, the only one wait_group.read 1 leaves
+        // running, always reads the other box.
+        uint32_t piece = 0;
+        auto load_x = [&](int tile, int col, uint8_t *box) {
             const int m0 = ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32;
-            bulk_wait_read_all();  // the box's previous store has read it
+            bulk_wait_read_all();  // every earlier store has read its box
             mbar_arrive_expect_tx(my_xbar, 4096);
-            tma_load_2d(staging + (warp - 2) * 4096, &tmC, my_xbar,
+            tma_load_2d(box, &tmC, my_xbar,
                         (tile % args.num_n_tiles) * BN + half * (BN / 2) + col, m0);
             x_pending = true;
         };
@@ -576,7 +585,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             constexpr int HW = BN / 2;
             const bool f32 = args.epi == kEpiResidF32 || args.epi == kEpiF32;
             const int pcols = f32 ? 32 : 64;
-            uint8_t *stg = staging + (warp - 2) * 4096;
+
             const int m0 = ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32;
             const bool slab = m0 < args.M;  // warp-uniform
             const int n_first = (tile % args.num_n_tiles) * BN + half * HW;
@@ -584,6 +593,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             t_acc += half * HW;
 #pragma unroll 1
             for (int p = 0; p < HW / pcols; ++p) {
+                uint8_t *stg = my_boxes + (piece & 1u) * 4096;
                 uint32_t w[32];  // this row's 128-byte piece as 8 chunks of 4 words
                 if (f32) {
                     float v[2][16];
@@ -599,7 +609,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                             for (int j = 0; j < 16; ++j) v[i][j] += r[i][j];
                     } else {
-                        if (resid_drain && slab && p > 0 && lane == 0) load_x(tile, p * pcols);
+                        if (resid_drain && slab && p > 0 && lane == 0) load_x(tile, p * pcols, stg);
                         __syncwarp();  // the warp-wide TMEM wait needs every lane here
                         tc_wait_ld();
                         if (!resid) {
@@ -667,8 +677,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         }
                     }
                 }
-                // The previous piece's store has finished reading the box.
-                if (lane == 0) bulk_wait_read_all();
+                // The store issued from this box two pieces ago has read it (the
+                // previous piece's store, from the other box, may still run).
+                if (lane == 0) bulk_wait_read_1();
                 __syncwarp();
                 uint8_t *row = stg + lane * 128;
 #pragma unroll
@@ -681,6 +692,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tma_store_2d(&tmC, stg, n_first + p * pcols, m0);
                     bulk_commit();
                 }
+                if (slab) ++piece;
                 __syncwarp();  // converged again before the next warp-wide TMEM load
             }
         };
@@ -694,7 +706,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 prefetch_l1(args.bias + (tile % args.num_n_tiles) * BN + half * (BN / 2) + lane * 4);
             if (resid_drain && lane == 0 &&  // first residual piece lands during the mainloop
                 ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32 < args.M)
-                load_x(tile, 0);
+                load_x(tile, 0, my_boxes + (piece & 1u) * 4096);
             __syncwarp();  // lane 0's residual load above is the only divergent step
             if (!mbar_wait_warp(tfull + acc, acc_phase, abort_v, lim)) {
                 ok = false;

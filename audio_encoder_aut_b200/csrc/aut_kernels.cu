@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
                                                     int chunk_base, const bf16 *__restrict__ w,
                                                     const bf16 *__restrict__ b,
                                                     bf16 *__restrict__ planes, int plane_rows,
+                                                    bf16 *__restrict__ planes2, int plane2_rows,
                                                     int C) {
     pdl_trigger();
     pdl_wait();
@@ -109,38 +110,25 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
             reinterpret_cast<uint4 *>(planes + (row * kP1Cols + col) * C)[co] =
                 make_uint4(0u, 0u, 0u, 0u);
         }
-}
-
-// Zero row and zero column of every chunk's rows of the four phase planes, and
-// (odd-column planes with `last_col`) their last column: the kernels that fill
-// the planes never write them.  Planes [4][plane_rows][cols][C], chunk_rows
-// rows per chunk, row 0 of a chunk and column 0 the zero borders.
-__global__ void __launch_bounds__(256) zero_plane_pads_kernel(bf16 *planes, int plane_rows,
-                                                              int chunk_rows, int cols,
-                                                              int last_col, int C) {
-    pdl_trigger();
-    pdl_wait();
-    const int cl = blockIdx.x, plane = blockIdx.y;
-    const int CP = C >> 1;
-    const size_t row0 = (size_t)plane * plane_rows + (size_t)cl * chunk_rows;
-    const int extra = (last_col && (plane & 1)) ? (chunk_rows - 1) : 0;
-    const int n = (cols + (chunk_rows - 1) + extra) * CP;
-    for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
-        const int e = idx / CP, cp = idx - e * CP;
-        size_t row;
-        int col;
-        if (e < cols) {
-            row = row0;
-            col = e;
-        } else if (e < cols + chunk_rows - 1) {
-            row = row0 + 1 + (e - cols);
-            col = 0;
-        } else {
-            row = row0 + 1 + (e - cols - (chunk_rows - 1));
-            col = cols - 1;
-        }
-        reinterpret_cast<uint32_t *>(planes + (row * cols + col) * C)[cp] = 0u;
+    // The zero borders of conv3's input planes (conv2's output, [4][.][kP2Cols][C])
+    // for this chunk, which conv2's epilogue never writes: this block clears
+    // column 0 and, in odd-column planes, the missing last column of plane rows
+    // 2 hg + 1 and 2 hg + 2; the first block also clears row 0.
+    const size_t chunk2_row0 = (size_t)cl * kP2Rows;
+    for (int idx = slice; idx < 4 * 2 * 2; idx += slices) {
+        const int plane = idx >> 2, r = 2 * hg + 1 + ((idx >> 1) & 1), side = idx & 1;
+        if (side == 1 && !(plane & 1)) continue;
+        const size_t row = (size_t)plane * plane2_rows + chunk2_row0 + r;
+        const int col = side ? kP2Cols - 1 : 0;
+        reinterpret_cast<uint4 *>(planes2 + (row * kP2Cols + col) * C)[co] = make_uint4(0u, 0u, 0u, 0u);
     }
+    if (hg == 0)
+        for (int idx = slice; idx < 4 * kP2Cols; idx += slices) {
+            const int plane = idx / kP2Cols, col = idx - plane * kP2Cols;
+            const size_t row = (size_t)plane * plane2_rows + chunk2_row0;
+            reinterpret_cast<uint4 *>(planes2 + (row * kP2Cols + col) * C)[co] =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
 }
 
 // -------------------------------------------------------------- layernorm --
@@ -474,20 +462,14 @@ int sm_count_cached() {
 
 cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int chunk_base,
                          int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
-                         int C, cudaStream_t st) {
+                         void *planes2, int plane2_rows, int C, cudaStream_t st) {
     if (n_chunks <= 0) return cudaSuccess;
+    static_assert(kC1Rows / 8 * 2 == kP2Rows - 1, "two conv3-input plane rows per conv1 block");
     return launch_pdl(conv1_kernel, dim3(n_chunks, kC1Rows / 8), dim3(256), 0, st, 1,
                       static_cast<const bf16 *>(feats), T_max, chunks, chunk_base,
                       static_cast<const bf16 *>(w), static_cast<const bf16 *>(b),
-                      static_cast<bf16 *>(planes), plane_rows, C);
-}
-
-cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int chunk_rows,
-                                   int cols, bool last_col, int C, cudaStream_t st) {
-    if (n_chunks <= 0) return cudaSuccess;
-    return launch_pdl(zero_plane_pads_kernel, dim3(n_chunks, 4), dim3(256), 0, st, 1,
-                      static_cast<bf16 *>(planes), plane_rows, chunk_rows, cols, last_col ? 1 : 0,
-                      C);
+                      static_cast<bf16 *>(planes), plane_rows, static_cast<bf16 *>(planes2),
+                      plane2_rows, C);
 }
 
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,

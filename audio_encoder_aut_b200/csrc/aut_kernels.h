@@ -79,11 +79,12 @@ struct UploadPayload {
     int32_t words[kWords];
 };
 
+// conv1 + GELU into conv2's input phase planes (`planes`, borders included);
+// also clears the zero borders of conv3's input planes (`planes2`) for the
+// same chunk slots.
 cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int chunk_base,
                          int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
-                         int C, cudaStream_t st);
-cudaError_t launch_zero_plane_pads(void *planes, int plane_rows, int n_chunks, int chunk_rows,
-                                   int cols, bool last_col, int C, cudaStream_t st);
+                         void *planes2, int plane2_rows, int C, cudaStream_t st);
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
                              float eps, cudaStream_t st, bool split = false);
 cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st);

@@ -126,6 +126,9 @@ AUT_DEV void tma_store_2d(const CUtensorMap *m, const void *src, int c0, int c1)
 AUT_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Every committed bulk store of this thread has finished reading shared memory.
 AUT_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Every committed bulk store of this thread but the most recent has finished
+// reading shared memory.
+AUT_DEV void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // Every committed bulk store of this thread has completed.
 AUT_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 AUT_DEV void prefetch_l1(const void *p) {

@@ -144,7 +144,7 @@ aut_status aut_encode(const aut_config *cfg, const aut_weights *prepared, const 
 /* Kernel kinds reported by aut_encode_traced. */
 typedef enum {
     AUT_K_UPLOAD = 0,    /* plan tables to the device */
-    AUT_K_ZERO_PADS = 1, /* zero borders of conv3's input planes */
+    AUT_K_ZERO_PADS = 1, /* (no longer launched: conv1 writes the planes' zero borders) */
     AUT_K_CONV1 = 2,
     AUT_K_CONV2 = 3,
     AUT_K_CONV3 = 4,

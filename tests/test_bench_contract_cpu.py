@@ -26,3 +26,17 @@ def test_reference_arm_prints_the_contract_line():
     assert d["config"]["windows"] == 2 and d["config"]["chunks"] == 3
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_gpus_flag_spawns_ranks_and_rank0_alone_prints():
+    """`--gpus 2` outside a launcher starts two ranks itself; on the reference
+    arm rank 0 alone runs and prints the one JSON line, rank 1 exits 0."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "0", "--gpus", "2"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["config"]["launch"].startswith("numpy oracle")
