@@ -8,12 +8,15 @@ import os
 import re
 from ctypes import POINTER, c_char_p, c_float, c_int32, c_size_t, c_void_p
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaut.so")
+# AUT_LIB=debug selects the bounds-checked build (libaut_debug.so, built by
+# `python -m audio_encoder_aut_b200.build --debug-bounds`).
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libaut_debug.so" if os.environ.get("AUT_LIB") == "debug" else "libaut.so")
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
                       "aut.h")
 
 AUT_OK, AUT_ERR_INVALID_ARG, AUT_ERR_UNSUPPORTED, AUT_ERR_WORKSPACE, AUT_ERR_CUDA, \
-    AUT_ERR_TIMEOUT = range(6)
+    AUT_ERR_TIMEOUT, AUT_ERR_BOUNDS = range(7)
 
 EPI_BF16, EPI_BF16_GELU, EPI_RESID_F32, EPI_F32 = 0, 1, 2, 3
 LINEAR_FAULT_INJECT, LINEAR_SINGLE_CTA, LINEAR_F16 = 1, 2, 4

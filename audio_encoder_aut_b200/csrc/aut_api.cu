@@ -12,6 +12,7 @@
 //     residual)
 //   final LN -> proj1 (GEMM + bias + GELU) -> proj2 (GEMM + bias) -> out (fp32)
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstring>
 
@@ -21,6 +22,16 @@
 namespace aut {
 
 namespace {
+
+// NVTX range over one stage of the forward (the stem, a layer, the projector),
+// for profilers; a host-side marker only, so it costs nothing on the device and
+// is recorded once when the forward is captured into a graph.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 constexpr unsigned long long kDefaultTimeoutNs = 4000ull * 1000ull * 1000ull;  // 4 s
 
@@ -165,6 +176,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
     const int n_ch = (int)p.chunks.size();
     const int G = c.L.group_chunks;
     if (n_ch == 0) return AUT_OK;
+    NvtxRange range("aut stem");
     const int4 *chunks = c.at<int4>(c.L.chunks);
     void *planes1 = c.at<void>(c.L.planes1);
     void *planes2 = c.at<void>(c.L.planes2);
@@ -173,7 +185,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
     for (int c0 = 0; c0 < n_ch; c0 += G) {
         const int g = std::min(G, n_ch - c0);
         AUT_TRY(cuda_status(launch_conv1(feats, T_max, chunks, c0, g, c.w->conv1_w, c.w->conv1_b,
-                                         planes1, p1_rows, planes2, p2_rows, C, c.st)));
+                                         planes1, p1_rows, planes2, p2_rows, C, c.st, c.status)));
         AUT_TRY(c.mark(AUT_K_CONV1));
         ConvLaunch k2{};
         k2.planes = planes1;
@@ -188,6 +200,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
         k2.bias = c.w->conv2_b;
         k2.epi = kEpiConvPlanes;
         k2.out = planes2;
+        k2.out_elems = (size_t)4 * p2_rows * kP2Cols * C;
         k2.dst_plane_rows = p2_rows;
         k2.dst_chunk_rows = kP2Rows;
         k2.dst_cols = kP2Cols;
@@ -206,6 +219,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
         k3.bias = c.w->conv3_b;
         k3.epi = kEpiConvFlat;
         k3.out = y3;
+        k3.out_elems = (size_t)G * kTokensPerChunk * kStemRows * C;
         AUT_TRY(gemm_status(launch_conv_gemm(k3, c.st)));
         AUT_TRY(c.mark(AUT_K_CONV3));
         LinearLaunch lo{};
@@ -213,6 +227,7 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
         lo.w = c.w->conv_out_w_fc;
         lo.bias = c.w->conv_out_b;
         lo.out = x0;
+        lo.out_elems = (size_t)p.total_tokens * d;
         lo.M = g * kTokensPerChunk;
         lo.N = d;
         lo.K = kStemRows * C;
@@ -238,7 +253,14 @@ aut_status run_encode(const Ctx &c, float *x, int T, int nW, int n_layers, void 
     void *xn = c.at<void>(c.L.xn), *qkv = c.at<void>(c.L.qkv), *attn = c.at<void>(c.L.attn),
          *ffn = c.at<void>(c.L.ffn);
     const int *cu = c.at<int>(c.L.cu);
+    static const char *const kLayerNames[] = {
+        "aut layer 0",  "aut layer 1",  "aut layer 2",  "aut layer 3",  "aut layer 4",
+        "aut layer 5",  "aut layer 6",  "aut layer 7",  "aut layer 8",  "aut layer 9",
+        "aut layer 10", "aut layer 11", "aut layer 12", "aut layer 13", "aut layer 14",
+        "aut layer 15", "aut layer 16", "aut layer 17", "aut layer 18", "aut layer 19",
+        "aut layer 20", "aut layer 21", "aut layer 22", "aut layer 23", "aut layer"};
     for (int l = 0; l < n_layers; ++l) {
+        NvtxRange range(kLayerNames[l < 24 ? l : 24]);
         const aut_layer_weights &lw = c.w->layers[l];
         AUT_TRY(cuda_status(launch_layernorm(x, lw.ln1_w, lw.ln1_b, xn, T, d, cfg->ln_eps, c.st)));
         AUT_TRY(c.mark(AUT_K_LAYERNORM));
@@ -259,6 +281,7 @@ aut_status run_encode(const Ctx &c, float *x, int T, int nW, int n_layers, void 
         AUT_TRY(linear(c, ffn, lw.fc2_w, lw.fc2_b, x, T, d, F, kEpiResidF32, AUT_K_FC2));
     }
     if (!out) return AUT_OK;
+    NvtxRange range("aut projector");
     // Projector operands as hi + lo bf16 pairs ([hi | lo] rows against K-repeated
     // weights): its two roundings would otherwise add as much error as a layer.
     AUT_TRY(cuda_status(

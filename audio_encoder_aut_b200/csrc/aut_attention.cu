@@ -111,7 +111,7 @@ __device__ __forceinline__ void local_window(const int2 *cache, const int *cu, i
 __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_qkv, __half *__restrict__ out, const int *__restrict__ cu,
     int n_windows, int heads, int d, float scale_log2e, int *status, int v_f16,
-    unsigned long long lim, int fault_inject) {
+    unsigned long long lim, int fault_inject, int T) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) window_attn_tc_kernel(
                     float o[32];
                     tmem_ld32(trow + kColO + ob * kHd + 32 * hh, o);
                     tc_wait_ld();
-                    if (row < len) {
+                    if (row < len && AUT_IN_BOUNDS(s0 + row < T, status)) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             uint32_t pk[4];
@@ -436,7 +436,7 @@ cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu
     return launch_pdl(window_attn_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, 1, tm,
                       static_cast<__half *>(out), cu_dev, n_windows, heads, d, scale_log2e, status,
                       v_f16 ? 1 : 0, timeout_ns ? timeout_ns : 4000ull * 1000ull * 1000ull,
-                      fault_inject);
+                      fault_inject, T);
 }
 
 }  // namespace aut

@@ -168,6 +168,7 @@ GemmStatus launch_linear(const LinearLaunch &L, cudaStream_t st) {
     args.epi = L.epi;
     args.bias = static_cast<const __nv_bfloat16 *>(L.bias);
     args.out = L.out;
+    args.out_elems = L.out_elems ? L.out_elems : (size_t)L.M * L.ldo;
     args.ldo = L.ldo;
     args.chunks = L.chunks;
     args.chunk_base = L.chunk_base;
@@ -229,6 +230,7 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     args.epi = L.epi;
     args.bias = static_cast<const __nv_bfloat16 *>(L.bias);
     args.out = L.out;
+    args.out_elems = L.out_elems;
     args.C = L.C;
     args.dst_plane_rows = L.dst_plane_rows;
     args.dst_chunk_rows = L.dst_chunk_rows;

@@ -48,6 +48,7 @@ struct GemmArgs {
     int epi;
     const __nv_bfloat16 *bias;  // [N] or nullptr
     void *out;
+    size_t out_elems;  // elements of the output buffer (bounds checks of debug builds)
     int ldo;
     int C;               // conv channels (conv epilogues)
     int dst_plane_rows;  // rows of one destination phase plane (kEpiConvPlanes)
@@ -738,6 +739,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (k == 1 && !two) break;
                     float(&v)[16] = k ? v1 : v0;
                     const int n0 = n_blk * BN + (k ? c1 : c0) * 16;
+                    const size_t end = dst_row + n0 + (args.epi == kEpiBf16GeluSplit ? args.N : 0) + 16;
+                    if (!AUT_IN_BOUNDS(end <= args.out_elems, args.status)) continue;
                     if (!resid) add_bias16(v, args.bias, n0);
                     switch (args.epi) {
                         case kEpiBf16:

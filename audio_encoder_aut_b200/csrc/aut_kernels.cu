@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
                                                     const bf16 *__restrict__ b,
                                                     bf16 *__restrict__ planes, int plane_rows,
                                                     bf16 *__restrict__ planes2, int plane2_rows,
-                                                    int C) {
+                                                    int C, int *status) {
     pdl_trigger();
     pdl_wait();
     const int cl = blockIdx.x, hg = blockIdx.y;
@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
         const int h = 8 * hg + hl;
         const int plane = (h & 1) * 2 + (wo & 1);
         const size_t row = (size_t)plane * plane_rows + chunk_row0 + (h >> 1) + 1;
+        if (!AUT_IN_BOUNDS(row < (size_t)4 * plane_rows && (wo >> 1) + 1 < kP1Cols, status)) continue;
         uint4 *dst = reinterpret_cast<uint4 *>(planes + (row * kP1Cols + (wo >> 1) + 1) * C) + co;
         *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ fea
         if (side == 1 && !(plane & 1)) continue;
         const size_t row = (size_t)plane * plane2_rows + chunk2_row0 + r;
         const int col = side ? kP2Cols - 1 : 0;
+        if (!AUT_IN_BOUNDS(row < (size_t)4 * plane2_rows, status)) continue;
         reinterpret_cast<uint4 *>(planes2 + (row * kP2Cols + col) * C)[co] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (hg == 0)
@@ -462,14 +464,14 @@ int sm_count_cached() {
 
 cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int chunk_base,
                          int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
-                         void *planes2, int plane2_rows, int C, cudaStream_t st) {
+                         void *planes2, int plane2_rows, int C, cudaStream_t st, int *status) {
     if (n_chunks <= 0) return cudaSuccess;
     static_assert(kC1Rows / 8 * 2 == kP2Rows - 1, "two conv3-input plane rows per conv1 block");
     return launch_pdl(conv1_kernel, dim3(n_chunks, kC1Rows / 8), dim3(256), 0, st, 1,
                       static_cast<const bf16 *>(feats), T_max, chunks, chunk_base,
                       static_cast<const bf16 *>(w), static_cast<const bf16 *>(b),
                       static_cast<bf16 *>(planes), plane_rows, static_cast<bf16 *>(planes2),
-                      plane2_rows, C);
+                      plane2_rows, C, status);
 }
 
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,

@@ -84,7 +84,8 @@ struct UploadPayload {
 // same chunk slots.
 cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int chunk_base,
                          int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
-                         void *planes2, int plane2_rows, int C, cudaStream_t st);
+                         void *planes2, int plane2_rows, int C, cudaStream_t st,
+                         int *status = nullptr);
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
                              float eps, cudaStream_t st, bool split = false);
 cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st);
@@ -121,6 +122,7 @@ struct LinearLaunch {
     const void *w;     // bf16 (fp16 with f16) [N, K]
     const void *bias;  // bf16 [N] or null
     void *out;
+    size_t out_elems = 0;  // elements of `out` (0: M * ldo)
     int M, N, K, ldo;
     int epi;           // GemmEpilogue
     // pack-tokens epilogue
@@ -149,6 +151,7 @@ struct ConvLaunch {
     const void *bias;    // bf16 [C]
     int epi;             // kEpiConvPlanes (conv2) or kEpiConvFlat (conv3)
     void *out;
+    size_t out_elems;    // elements of `out`
     int dst_plane_rows, dst_chunk_rows, dst_cols;  // kEpiConvPlanes destination geometry
     int *status;
     unsigned long long timeout_ns;

@@ -110,6 +110,7 @@ extern "C" const char *aut_status_string(aut_status s) {
         case AUT_ERR_WORKSPACE: return "workspace or destination too small";
         case AUT_ERR_CUDA: return "CUDA error";
         case AUT_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case AUT_ERR_BOUNDS: return "device index out of bounds (debug build)";
     }
     return "unknown status";
 }

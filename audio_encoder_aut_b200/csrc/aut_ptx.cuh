@@ -14,6 +14,21 @@ namespace aut {
 // Status codes written by kernels into a device status word (same values as
 // aut_status in include/aut.h).
 constexpr int kDevTimeout = 5;
+constexpr int kDevBounds = 6;
+
+// Debug builds (-DAUT_DEBUG_BOUNDS, libaut_debug.so) check the computed global
+// addresses of the kernels that do not go through TMA: a failed check writes
+// AUT_ERR_BOUNDS to the status word and the access is skipped, nothing traps.
+// Release builds compile the checks away.
+#ifdef AUT_DEBUG_BOUNDS
+#define AUT_IN_BOUNDS(cond, status) ::aut::bounds_ok((cond), (status))
+#else
+#define AUT_IN_BOUNDS(cond, status) true
+#endif
+__device__ __forceinline__ bool bounds_ok(bool ok, int *status) {
+    if (!ok && status) atomicCAS(status, 0, kDevBounds);
+    return ok;
+}
 
 AUT_DEV uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

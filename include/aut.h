@@ -43,7 +43,10 @@ typedef enum {
     AUT_ERR_UNSUPPORTED = 2,  /* configuration outside what the kernels implement */
     AUT_ERR_WORKSPACE = 3,    /* workspace or destination buffer too small */
     AUT_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
-    AUT_ERR_TIMEOUT = 5       /* a device pipeline wait ran out of time (from aut_check) */
+    AUT_ERR_TIMEOUT = 5,      /* a device pipeline wait ran out of time (from aut_check) */
+    AUT_ERR_BOUNDS = 6        /* debug builds (libaut_debug.so, -DAUT_DEBUG_BOUNDS): a kernel
+                               * computed an address outside its buffer and skipped the
+                               * access (from aut_check) */
 } aut_status;
 
 /* Encoder hyper-parameters; field meaning follows AuTEncoderConfig on the
