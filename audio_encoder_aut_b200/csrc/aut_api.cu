@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <cstring>
 
 #include "aut_internal.h"
@@ -151,11 +152,35 @@ aut_status linear(const Ctx &c, const void *a, const void *w, const void *b, voi
     return c.mark(kind);
 }
 
-// The chunk table and cu_seqlens lie next to each other in the workspace
-// (chunks, padding, cu); one upload writes the whole span.
+// cu_seqlens followed by the window table the tensor-core attention walks:
+// (first token, length) per window, longest first, ties in window order, so
+// that its grid stride gives every CTA a similar mix of long and short
+// windows.  The table starts on an even word of the region (8-byte aligned).
+void append_windows(std::vector<int32_t> &words, const std::vector<int32_t> &cu) {
+    const int nW = (int)cu.size() - 1;
+    words.insert(words.end(), cu.begin(), cu.end());
+    if (words.size() & 1) words.push_back(0);
+    std::vector<int> order(nW);
+    for (int i = 0; i < nW; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+        return cu[a + 1] - cu[a] > cu[b + 1] - cu[b];
+    });
+    for (int w : order) {
+        words.push_back(cu[w]);
+        words.push_back(cu[w + 1] - cu[w]);
+    }
+}
+
+// Device address of the window table behind cu_seqlens (append_windows).
+const int2 *window_table(const Ctx &c, int nW) {
+    return reinterpret_cast<const int2 *>(c.at<int32_t>(c.L.cu) + nW + 1 + ((nW + 1) & 1));
+}
+
+// The chunk table, cu_seqlens and the window table lie next to each other in
+// the workspace (chunks, padding, cu, windows); one upload writes the span.
 aut_status upload_plan(const Ctx &c, const Plan &p) {
     const size_t cu_word = (c.L.cu - c.L.chunks) / 4;
-    std::vector<int32_t> words(cu_word + p.cu_seqlens.size(), 0);
+    std::vector<int32_t> words(cu_word, 0);
     size_t i = 0;
     for (const ChunkInfo &ci : p.chunks) {
         words[i++] = ci.request;
@@ -163,7 +188,7 @@ aut_status upload_plan(const Ctx &c, const Plan &p) {
         words[i++] = ci.valid_frames;
         words[i++] = ci.token0;
     }
-    std::copy(p.cu_seqlens.begin(), p.cu_seqlens.end(), words.begin() + cu_word);
+    append_windows(words, p.cu_seqlens);
     AUT_TRY(cuda_status(launch_upload(words.data(), words.size(), c.at<int32_t>(c.L.chunks), c.st)));
     return c.mark(AUT_K_UPLOAD);
 }
@@ -270,7 +295,7 @@ aut_status run_encode(const Ctx &c, float *x, int T, int nW, int n_layers, void 
         AUT_TRY(linear(c, xn, lw.qkv_w, lw.qkv_b, qkv, T, 3 * d, d, kEpiBf16, AUT_K_QKV, 0, false,
                        v_f16 ? 2 * d : 1 << 30));
         AUT_TRY(cuda_status(launch_window_attention(qkv, attn, cu, nW, d, cfg->heads, c.st, T,
-                                                    c.status, v_f16)));
+                                                    c.status, v_f16, 0, 0, window_table(c, nW))));
         AUT_TRY(c.mark(AUT_K_ATTENTION));
         // fp16 attention output against the fp16 copy of o_w
         const void *o_w16 = static_cast<const uint8_t *>(c.w->o_w_f16) + (size_t)l * d * d * 2;
@@ -329,7 +354,7 @@ WorkspaceLayout workspace_layout(const aut_config *c, int64_t T, int64_t nW, int
     const size_t d = c->d_model, F = c->ffn, C = c->conv_ch;
     L.status = r.take(256);
     L.chunks = r.take((size_t)std::max<int64_t>(n_ch, 1) * 16);
-    L.cu = r.take((size_t)(nW + 1) * 4);
+    L.cu = r.take((size_t)(3 * nW + 2) * 4);  // cu_seqlens, one padding word, window table
     L.x = r.take((size_t)T * d * 4);
     // The stem buffers and the layer buffers are never live together: overlay them.
     const size_t base = r.off;
@@ -472,8 +497,9 @@ extern "C" aut_status aut_encode_packed(const aut_config *cfg, const aut_weights
     Ctx c;
     AUT_TRY(make_ctx(cfg, prepared, workspace, ws_bytes, p, reinterpret_cast<cudaStream_t>(stream), &c));
     if (total_tokens == 0) return AUT_OK;
-    AUT_TRY(cuda_status(launch_upload(p.cu_seqlens.data(), p.cu_seqlens.size(),
-                                      c.at<int32_t>(c.L.cu), c.st)));
+    std::vector<int32_t> words;
+    append_windows(words, p.cu_seqlens);
+    AUT_TRY(cuda_status(launch_upload(words.data(), words.size(), c.at<int32_t>(c.L.cu), c.st)));
     return run_encode(c, static_cast<float *>(hidden), total_tokens, num_windows, n_layers, out);
 }
 

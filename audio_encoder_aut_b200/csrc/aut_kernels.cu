@@ -519,12 +519,13 @@ cudaError_t run_window_attention(const bf16 *q, __half *o, const int *cu_dev, in
 
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                     int d, int heads, cudaStream_t st, int T, int *status,
-                                    bool v_f16, unsigned long long timeout_ns, int fault_inject) {
+                                    bool v_f16, unsigned long long timeout_ns, int fault_inject,
+                                    const int2 *wins) {
     if (n_windows <= 0) return cudaSuccess;
     const int hd = d / heads;
     if (window_attention_uses_tc(d, heads, T))
         return launch_window_attention_tc(qkv, out, cu_dev, n_windows, d, heads, T, status, st,
-                                          v_f16, timeout_ns, fault_inject);
+                                          v_f16, timeout_ns, fault_inject, wins);
     if (v_f16 || fault_inject) return cudaErrorInvalidValue;
     const float scale_log2e = 1.4426950408889634f / sqrtf((float)hd);
     const bf16 *q = static_cast<const bf16 *>(qkv);

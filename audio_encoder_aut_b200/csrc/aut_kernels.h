@@ -92,10 +92,14 @@ cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStr
 cudaError_t launch_to_f16(const void *src, void *dst, size_t n, cudaStream_t st);
 // v_f16: the v third of qkv already holds fp16 (the qkv GEMM wrote it so); only
 // the head_dim-64 tensor-core path (T > 0) accepts it.
+// wins (device, optional, tensor-core path only): the windows as (first token,
+// length) pairs, longest first; the kernel walks its (window, head) tiles in
+// that order.  Null: cu_seqlens order.
 cudaError_t launch_window_attention(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                     int d, int heads, cudaStream_t st, int T = -1,
                                     int *status = nullptr, bool v_f16 = false,
-                                    unsigned long long timeout_ns = 0, int fault_inject = 0);
+                                    unsigned long long timeout_ns = 0, int fault_inject = 0,
+                                    const int2 *wins = nullptr);
 // Whether launch_window_attention takes the tensor-core path.
 inline bool window_attention_uses_tc(int d, int heads, int T) { return d / heads == 64 && T > 0; }
 // tcgen05 variant for head_dim 64 (aut_attention.cu); T = rows of qkv.
@@ -104,7 +108,7 @@ inline bool window_attention_uses_tc(int d, int heads, int T) { return d / heads
 cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu_dev, int n_windows,
                                        int d, int heads, int T, int *status, cudaStream_t st,
                                        bool v_f16 = false, unsigned long long timeout_ns = 0,
-                                       int fault_inject = 0);
+                                       int fault_inject = 0, const int2 *wins = nullptr);
 // bf16 tensor map with 128-byte swizzle (aut_gemm.cu): dims innermost first,
 // strides in bytes for dims 1.., box in elements.
 bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,

@@ -56,14 +56,19 @@ AUT_DEV void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
 AUT_DEV void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
+// A waiting thread is suspended (up to kWaitSuspendNs, or until the phase
+// completes) instead of polling: a polling warp takes issue slots from the
+// warps on its scheduler that have work, such as a GEMM's MMA issuer and
+// epilogue.
+constexpr uint32_t kWaitSuspendNs = 2000;
 AUT_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kWaitSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -81,6 +86,20 @@ AUT_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint
         if (abort && *abort) return false;
         if (global_timer_ns() - t0 > limit_ns) return false;
     }
+}
+
+// Non-blocking: whether the phase with the given parity has completed
+// (acquire semantics, as a successful wait).
+AUT_DEV bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 q, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
 }
 
 // mbar_wait for a whole converged warp, with one answer for every lane: each
@@ -108,10 +127,10 @@ AUT_DEV bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns
         uint32_t ok;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}\n"
             : "=r"(ok)
-            : "r"(smem_addr(bar)), "r"(parity)
+            : "r"(smem_addr(bar)), "r"(parity), "r"(kWaitSuspendNs)
             : "memory");
         if (ok) return true;
         if (global_timer_ns() - t0 > limit_ns) return false;
@@ -357,6 +376,23 @@ AUT_DEV float2 fmul2(float2 a, float2 b) {
     unsigned long long d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
     return f2_from(d);
+}
+
+AUT_DEV float2 fadd2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return f2_from(d);
+}
+AUT_DEV float2 fsub2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return f2_from(d);
+}
+// max(a, b, c) in one instruction.
+AUT_DEV float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // gelu_fast on two values, the polynomial and scaling in packed fp32x2.
