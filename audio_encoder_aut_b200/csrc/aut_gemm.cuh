@@ -347,8 +347,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     // failure; the bound here is well past that, so this spin
                     // cannot run out first and settle a phase it still waits on.
                     volatile int *mx = mma_exit;
-                    while (!*mx && global_timer_ns() - t0 < 4 * lim) {
-                    }
+                    while (!*mx && global_timer_ns() - t0 < 4 * lim)
+                        __nanosleep(128);  // the last tile's MMAs and drain use the issue slots
                     t0 = global_timer_ns();
                     const bool got = mbar_wait_cluster(exit_bar, 0, left());
 #pragma unroll
