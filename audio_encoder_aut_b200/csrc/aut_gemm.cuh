@@ -529,53 +529,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             }
         };
-        // Single-tile residual GEMMs: accumulator `acc` <- x + bias over this
-        // thread's row and the columns this warp drains.
-        auto preload = [&](int tile, int acc, bool rel) {
-            __syncwarp();  // TMEM stores are warp-wide
-            bool valid;
-            size_t dst_row;
-            int pos_row;
-            locate(tile, valid, dst_row, pos_row);
-            const int n_base = (tile % args.num_n_tiles) * BN;
-            const float *xp = reinterpret_cast<const float *>(args.out) + dst_row + n_base;
-            const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-            // The chunks this warp drains (so that it only ever overwrites what it
-            // has itself drained, and reads back only what it has itself written):
-            // a contiguous half of the columns for the TMA drain, else alternate
-            // 16-column chunks.
-            const int c_first = args.tma_out ? half * (NC / 2) : half;
-            const int c_step = args.tma_out ? 1 : 2;
-            const int c_count = args.tma_out ? NC / 2 : (NC - half + 1) / 2;
+        // Single-tile residual GEMMs (TMA-store epilogue): accumulator `acc` <-
+        // x + bias over this warp's 32 rows and its half of the columns, so that
+        // the drain adds acc + (x + bias).  x comes in by TMA through the warp's
+        // two staging boxes, 64 columns (two 128-byte boxes) per round, while
+        // the MMAs run.
+        auto preload = [&](int tile, int acc) {
+            constexpr int HW = BN / 2;
+            const int m0 = ((tile / args.num_n_tiles) * CG + (int)rank) * 128 + quad * 32;
+            const bool slab = m0 < args.M;  // warp-uniform
+            const int n_first = (tile % args.num_n_tiles) * BN + half * HW;
+            const uint32_t t_addr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN + half * HW;
 #pragma unroll 1
-            for (int i0 = 0; i0 < c_count; i0 += 4) {  // four chunks of loads in flight
-                float v[4][16];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c_first + (i0 + u) * c_step;
-                    if (i0 + u < c_count) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 e = valid ? reinterpret_cast<const float4 *>(xp + c * 16)[q]
-                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-                            v[u][4 * q] = e.x;
-                            v[u][4 * q + 1] = e.y;
-                            v[u][4 * q + 2] = e.z;
-                            v[u][4 * q + 3] = e.w;
-                        }
-                    }
+            for (int c0 = 0; c0 < HW; c0 += 64) {
+                const int nb = HW - c0 >= 64 ? 2 : 1;  // boxes this round (warp-uniform)
+                if (slab && lane == 0) {
+                    mbar_arrive_expect_tx(my_xbar, nb * 4096);
+                    for (int b = 0; b < nb; ++b)
+                        tma_load_2d(my_boxes + b * 4096, &tmC, my_xbar, n_first + c0 + 32 * b, m0);
+                    x_pending = true;
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c_first + (i0 + u) * c_step;
-                    if (i0 + u < c_count) {
-                        add_bias16(v[u], args.bias, n_base + c * 16);
-                        tmem_st16(t_addr + c * 16, v[u]);
+                __syncwarp();
+                if (slab) {
+                    if (!mbar_wait_warp(my_xbar, xph, abort_v, lim)) {
+                        ok = false;
+                        gemm_signal_abort(args, abort_v);
+                        return;
                     }
+                    x_pending = false;
+                    xph ^= 1u;
                 }
+                for (int b = 0; b < nb; ++b) {
+                    float xr[2][16];
+                    const uint8_t *row = my_boxes + b * 4096 + lane * 128;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 x4 = slab ? *reinterpret_cast<const float4 *>(
+                                                     row + ((j ^ (lane & 7)) << 4))
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                        float *q = &xr[j >> 2][(j & 3) * 4];
+                        q[0] = x4.x;
+                        q[1] = x4.y;
+                        q[2] = x4.z;
+                        q[3] = x4.w;
+                    }
+                    add_bias16(xr[0], args.bias, n_first + c0 + 32 * b);
+                    add_bias16(xr[1], args.bias, n_first + c0 + 32 * b + 16);
+                    tmem_st16(t_addr + c0 + 32 * b, xr[0]);
+                    tmem_st16(t_addr + c0 + 32 * b + 16, xr[1]);
+                }
+                // These reads of the boxes come before the next round's TMA writes.
+                fence_proxy_async_smem();
+                __syncwarp();
             }
             tc_wait_st();
-            if (rel) release(acc);
         };
 
         // Drain through shared memory: this warp's 32 rows x BN / 2 columns go
@@ -698,7 +705,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         };
 
-        if (resid_once && group < total_tiles) preload(group, 1, false);
+        if (resid_once && group < total_tiles) preload(group, 1);
         int it = 0;
         for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
             const int acc = it & 1;
