@@ -26,7 +26,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
               "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include"), "-I", CSRC]
 SOURCES = ["aut_plan.cpp", "aut_kernels.cu", "aut_gemm.cu", "aut_attention.cu", "aut_api.cu",
-           "aut_noalloc.cu", "aut_logmel.cu", "aut_inject.cu"]
+           "aut_noalloc.cu", "aut_logmel.cu", "aut_inject.cu", "aut_conv1.cu"]
 
 
 def nvcc() -> str:

@@ -209,8 +209,13 @@ aut_status run_frontend(const Ctx &c, const Plan &p, const void *feats, int T_ma
     const int p1_rows = G * kP1Rows, p2_rows = G * kP2Rows;
     for (int c0 = 0; c0 < n_ch; c0 += G) {
         const int g = std::min(G, n_ch - c0);
-        AUT_TRY(cuda_status(launch_conv1(feats, T_max, chunks, c0, g, c.w->conv1_w, c.w->conv1_b,
-                                         planes1, p1_rows, planes2, p2_rows, C, c.st, c.status)));
+        if (conv1_tc_supported(C))
+            AUT_TRY(cuda_status(launch_conv1_tc(feats, T_max, chunks, c0, g, c.w->conv1_w,
+                                                c.w->conv1_b, planes1, p1_rows, planes2, p2_rows, C,
+                                                c.st, c.status, kDefaultTimeoutNs)));
+        else
+            AUT_TRY(cuda_status(launch_conv1(feats, T_max, chunks, c0, g, c.w->conv1_w, c.w->conv1_b,
+                                             planes1, p1_rows, planes2, p2_rows, C, c.st, c.status)));
         AUT_TRY(c.mark(AUT_K_CONV1));
         ConvLaunch k2{};
         k2.planes = planes1;

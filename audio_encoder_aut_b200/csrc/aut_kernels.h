@@ -86,6 +86,14 @@ cudaError_t launch_conv1(const void *feats, int T_max, const int4 *chunks, int c
                          int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
                          void *planes2, int plane2_rows, int C, cudaStream_t st,
                          int *status = nullptr);
+// conv1 + GELU on the tensor cores (aut_conv1.cu): the same output as
+// launch_conv1, conv2's input planes and both plane sets' zero borders, for
+// C a multiple of 32 in [64, 512].
+bool conv1_tc_supported(int C);
+cudaError_t launch_conv1_tc(const void *feats, int T_max, const int4 *chunks, int chunk_base,
+                            int n_chunks, const void *w, const void *b, void *planes, int plane_rows,
+                            void *planes2, int plane2_rows, int C, cudaStream_t st, int *status,
+                            unsigned long long timeout_ns = 0);
 cudaError_t launch_layernorm(const float *x, const void *g, const void *b, void *y, int T, int d,
                              float eps, cudaStream_t st, bool split = false);
 cudaError_t launch_duplicate_k(const void *src, void *dst, int N, int K, cudaStream_t st);
