@@ -25,7 +25,8 @@ using bf16 = __nv_bfloat16;
 //
 // Block (chunk, 8 output rows); each thread computes eight channels (packed
 // fp32x2 arithmetic) for a strided set of positions, so a warp writes 32
-// consecutive 16-byte channel octets.
+// consecutive 16-byte channel octets.  This CUDA-core version serves the
+// channel counts the tensor-core conv1 (aut_conv1.cu) does not take.
 __global__ void __launch_bounds__(256) conv1_kernel(const bf16 *__restrict__ feats, int T_max,
                                                     const int4 *__restrict__ chunks,
                                                     int chunk_base, const bf16 *__restrict__ w,
