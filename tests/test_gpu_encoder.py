@@ -109,6 +109,25 @@ def test_asr06b_nonlinear_stem():
                                                   with_positions=False), "stem x25")
 
 
+@pytest.mark.parametrize("C", [64, 192, 240, 256, 384, 512])
+def test_stem_channel_counts(C):
+    """The stem at other conv widths: C = 64 .. 512 on the tensor-core conv1
+    (one or two blocks per group, no overlap or an overlapping last block,
+    N = C / 2 per MMA up to 256), C = 240 on the CUDA-core conv1; partial last
+    chunks; GELUs in their non-linear range (conv weights x 25)."""
+    import dataclasses
+    cfg = dataclasses.replace(S.TINY, downsample_hidden_size=C)
+    w = S.weights(cfg, conv_scale=25.0)
+    enc = Encoder(cfg, w, 0)
+    lens = [237, 1000, 450]
+    feats = S.features(lens)
+    h = enc.frontend(enc.features_to_device(feats), lens, with_positions=False)
+    torch.cuda.synchronize()
+    assert enc.check() == A.AUT_OK
+    assert_rows_close(h.cpu().numpy(), O.frontend(cfg, w, feats, lens, np.float32,
+                                                  with_positions=False), f"stem C={C}")
+
+
 def _sampled_windows(cfg, w, enc, lens, picks):
     """GPU on the whole batch; oracle on each picked (request, window) alone."""
     feats = S.features(lens)
