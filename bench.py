@@ -107,6 +107,18 @@ def layer_gemm_operand_bytes(cfg, T):
     return (qkv + o + fc1 + fc2) / 4
 
 
+def memory_kernel_bytes(cfg, T, n_chunks):
+    """Algorithmic bytes per step of the kernels measured against HBM bandwidth:
+    window attention reads q, k, v (6 d B) and writes O (2 d B) per token per
+    layer; each layer LayerNorm reads 4 d B and writes 2 d B per token, the final
+    one writes [hi | lo] (4 d B); conv1 reads the chunk's mel tile and writes its
+    64 x 50 x C bf16 output."""
+    d, L, C = cfg.d_model, cfg.encoder_layers, cfg.downsample_hidden_size
+    return {"attention": L * 8 * d * T,
+            "layernorm": 2 * L * 6 * d * T + 8 * d * T,
+            "conv1": n_chunks * (64 * 50 * C * 2 + 128 * 100 * 2)}
+
+
 # ---------------------------------------------------------------- clocks ----
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons sampled through NVML every 5 ms
@@ -361,6 +373,12 @@ def our_arm(args, rank, world, local_rank):
                        for k in kflops if k in kind_ms and kind_ms[k] > 0 and k in A.GEMM_KINDS}
     all_gemm = sum(kflops[k] for k in A.GEMM_KINDS if k in kflops)
     all_gemm_ms = sum(kind_ms[k] for k in A.GEMM_KINDS if k in kind_ms)
+    # The other kernels against HBM bandwidth: algorithmic bytes / event-timed time.
+    mem_bytes = memory_kernel_bytes(cfg, T, nch)
+    memory_kernels = {k: {"gb_per_s": round(b / (kind_ms[k] / 1e3) / 1e9, 1),
+                          "frac_hbm": round(b / (kind_ms[k] / 1e3) / 1e9 / hbm, 3),
+                          "mb_per_step": round(b / 1e6, 2)}
+                      for k, b in mem_bytes.items() if kind_ms.get(k, 0) > 0}
 
     # End to end through the public API: every step copies its features in from
     # pinned host memory and its fp32 result back out; the copies of steps
@@ -424,7 +442,9 @@ def our_arm(args, rank, world, local_rank):
                                          "o_proj, fc1, fc2)",
                          "algorithmic_bytes_per_launch": layer_gemm_operand_bytes(cfg, T),
                          "per_gemm": per_kind_tflops,
-                         "all_gemms_frac": all_gemm / (all_gemm_ms / 1e3) / 1e12 / pk},
+                         "all_gemms_frac": all_gemm / (all_gemm_ms / 1e3) / 1e12 / pk,
+                         "memory_kernels": memory_kernels,
+                         "hbm_peak_gbs": hbm, "hbm_peak_source": pk_src},
             "kernel_ms_per_step": {k: round(v, 4) for k, v in sorted(kind_ms.items(), key=lambda x: -x[1])},
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": h_feats.numel() * h_feats.element_size(),
