@@ -89,6 +89,7 @@ GemmStatus dispatch(int bn, int cg, const CUtensorMap &ta, const CUtensorMap &tb
             case 192: return run<192, 2>(ta, tb, tc, args, st);
             case 240: return run<240, 2>(ta, tb, tc, args, st);
             case 256: return run<256, 2>(ta, tb, tc, args, st);
+            case 480: return run<480, 2>(ta, tb, tc, args, st);  // two N = 240 MMAs per K step
             default: return GemmStatus::kBadShape;
         }
     }
@@ -202,6 +203,11 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     if (!aligned16(L.planes) || !aligned16(L.w_tap) || !aligned16(L.out) || !aligned16(L.bias))
         return GemmStatus::kBadShape;
     const int cg = (!L.single_cta && pair_ok(bn)) ? 2 : 1;
+    // C = 480 on CTA pairs: one tile covers all 480 output channels as two
+    // N = 240 MMAs per K step, so each SM loads its A tile once for 480
+    // channels instead of twice for 240 (the conv mainloop is bound by the
+    // operand bytes an SM takes in).
+    const int tile_n = (cg == 2 && bn == 240 && L.C == 480) ? 480 : bn;
     const long rows_total = (long)L.chunks * L.chunk_rows;
     CUtensorMap ta, tb;
     const cuuint64_t da[4] = {(cuuint64_t)L.C, (cuuint64_t)L.cols_in, (cuuint64_t)rows_total, 4};
@@ -219,7 +225,7 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     args.N = L.C;
     const long slot_rows = (long)L.rows_per_tile * cg;
     args.num_m_tiles = (int)((rows_total + slot_rows - 1) / slot_rows);
-    args.num_n_tiles = L.C / bn;
+    args.num_n_tiles = L.C / tile_n;
     args.conv = 1;
     args.conv_rows = L.rows_per_tile;
     args.conv_cols = L.out_cols;
@@ -237,7 +243,7 @@ GemmStatus launch_conv_gemm(const ConvLaunch &L, cudaStream_t st) {
     args.dst_cols = L.dst_cols;
     args.status = L.status;
     args.timeout_ns = L.timeout_ns;
-    return dispatch(bn, cg, ta, tb, tb, args, st);  // no TMA-store epilogue
+    return dispatch(tile_n, cg, ta, tb, tb, args, st);  // no TMA-store epilogue
 }
 
 }  // namespace aut

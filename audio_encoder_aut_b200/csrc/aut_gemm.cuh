@@ -72,11 +72,19 @@ struct GemmArgs {
 
 // BN: tile width of one MMA (N).  CG: CTAs per MMA (1, or 2 for a CTA pair
 // whose MMA is M = 256: each CTA holds 128 rows of A and BN / 2 rows of B).
+// A tile wider than one MMA (BN > 256) is two MMAs of BN / 2 per K step into
+// one accumulator of BN columns: the A operand then serves twice the columns
+// per byte an SM takes in, and the second accumulator (which would hide a
+// tile's drain behind the next tile's MMAs) no longer fits in tensor memory.
 template <int BN, int CG>
 struct GemmCfg {
     static constexpr int BM = 128, BK = 64;
+    static constexpr int NSPLIT = BN > 256 ? 2 : 1;  // MMAs per K step
+    static constexpr int MMA_N = BN / NSPLIT;
+    static constexpr int ACCS = NSPLIT == 1 ? 2 : 1;  // accumulators in tensor memory
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_ROWS = BN / CG;
+    static constexpr int B_SPLIT_ROWS = MMA_N / CG;  // B rows per MMA in this CTA
     static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     // Output staging for the TMA-store epilogue: two boxes of 32 rows x 128
@@ -90,16 +98,16 @@ struct GemmCfg {
     static constexpr int STAGES_FIT =
         (SMEM_LIMIT - 1024 - STAGING_BYTES - BAR_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-    static constexpr int TMEM_COLS = (2 * BN <= 32)    ? 32
-                                     : (2 * BN <= 64)  ? 64
-                                     : (2 * BN <= 128) ? 128
-                                     : (2 * BN <= 256) ? 256
-                                                       : 512;
+    static constexpr int TMEM_COLS = (ACCS * BN <= 32)    ? 32
+                                     : (ACCS * BN <= 64)  ? 64
+                                     : (ACCS * BN <= 128) ? 128
+                                     : (ACCS * BN <= 256) ? 256
+                                                          : 512;
     static constexpr int SMEM_BYTES =
         1024 /*alignment slack*/ + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
     static_assert(STAGES >= 3, "at least three operand stages");
-    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
-    static_assert(B_ROWS % 8 == 0, "each CTA holds whole 8-row swizzle atoms of B");
+    static_assert(MMA_N % 16 == 0 && MMA_N >= 16 && MMA_N <= 256 && ACCS * BN <= 512, "UMMA N");
+    static_assert(B_SPLIT_ROWS % 8 == 0, "each CTA holds whole 8-row swizzle atoms of B");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay aligned");
 };
 
@@ -246,21 +254,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (rank == 0) mbar_arrive_expect_tx(full + stage, CG * cta_bytes);
             };
             // Weights (B): k-block kb of the tile whose B rows start at b_row.
+            // With two MMAs per K step, this CTA's B rows of each MMA come from
+            // their own place in the weights (one box each, B_SPLIT_ROWS rows).
             auto load_b = [&](int stage, int kb, int b_row) {
-                uint8_t *b_dst = sB + stage * Cfg::B_BYTES;
-                if (!args.conv) {
-                    if constexpr (CG == 2)
-                        tma_load_2d_pair(b_dst, &tmB, map_to_rank(full + stage, 0), kb * 64, b_row);
-                    else
-                        tma_load_2d(b_dst, &tmB, full + stage, kb * 64, b_row);
-                } else {
-                    const int tap = kb / args.conv_cblocks;
-                    const int cb = kb - tap * args.conv_cblocks;
-                    if constexpr (CG == 2)
-                        tma_load_3d_pair(b_dst, &tmB, map_to_rank(full + stage, 0), cb * 64, tap,
-                                         b_row);
-                    else
-                        tma_load_3d(b_dst, &tmB, full + stage, cb * 64, tap, b_row);
+#pragma unroll
+                for (int h = 0; h < Cfg::NSPLIT; ++h) {
+                    uint8_t *b_dst = sB + stage * Cfg::B_BYTES + h * Cfg::B_SPLIT_ROWS * 128;
+                    const int row = b_row + h * Cfg::MMA_N;
+                    if (!args.conv) {
+                        if constexpr (CG == 2)
+                            tma_load_2d_pair(b_dst, &tmB, map_to_rank(full + stage, 0), kb * 64, row);
+                        else
+                            tma_load_2d(b_dst, &tmB, full + stage, kb * 64, row);
+                    } else {
+                        const int tap = kb / args.conv_cblocks;
+                        const int cb = kb - tap * args.conv_cblocks;
+                        if constexpr (CG == 2)
+                            tma_load_3d_pair(b_dst, &tmB, map_to_rank(full + stage, 0), cb * 64, tap,
+                                             row);
+                        else
+                            tma_load_3d(b_dst, &tmB, full + stage, cb * 64, tap, row);
+                    }
                 }
             };
             // Activations (A): k-block kb of the tile at 128-row slot m_slot.
@@ -299,7 +313,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int tile = group; ok && tile < total_tiles; tile += n_groups) {
                 const int n_blk = tile % args.num_n_tiles, m_blk = tile / args.num_n_tiles;
                 const int m_slot = m_blk * CG + (int)rank;  // this CTA's 128-row slot
-                const int b_row = n_blk * BN + (int)rank * Cfg::B_ROWS;
+                const int b_row = n_blk * BN + (int)rank * Cfg::B_SPLIT_ROWS;
                 for (int kb = 0; kb < args.num_k_blocks; ++kb) {
                     if (!mbar_wait(empty + stage, phase ^ 1u, abort_v, lim)) {
                         ok = false;
@@ -371,15 +385,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // -------------------------------------------------- MMA issuer --
-            const uint32_t idesc =
-                args.f16 ? idesc_f16_f32(128 * CG, BN) : idesc_bf16_f32(128 * CG, BN);
+            const uint32_t idesc = args.f16 ? idesc_f16_f32(128 * CG, Cfg::MMA_N)
+                                            : idesc_bf16_f32(128 * CG, Cfg::MMA_N);
             constexpr uint16_t kPair = 0x3;
             int stage = 0, it = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = group; ok && tile < total_tiles; tile += n_groups, ++it) {
-                const int acc = it & 1;
-                const uint32_t acc_phase = (it >> 1) & 1;
+                const int acc = it % Cfg::ACCS;
+                const uint32_t acc_phase = (uint32_t)(it / Cfg::ACCS) & 1u;
                 // Wait for the epilogue to have drained the accumulator (the
                 // phase before the first use counts as complete).
                 if (!mbar_wait(tempty + acc, acc_phase ^ 1u, abort_v, lim)) {
@@ -395,7 +409,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     tc_fence_after();
                     const uint64_t a_desc = smem_desc_sw128(sA + stage * Cfg::A_BYTES);
-                    const uint64_t b_desc = smem_desc_sw128(sB + stage * Cfg::B_BYTES);
                     // A convolution's last channel block of each tap may be partly
                     // past C (zero fill): only its K steps that hold channels run.
                     int ksteps = 4;
@@ -405,15 +418,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (left < 64) ksteps = (left + 15) >> 4;
                     }
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {  // K = 16 per MMA: +32 bytes in the row
-                        if (kk >= ksteps) break;
-                        const uint32_t accumulate = (kb | kk) != 0;
-                        if constexpr (CG == 2)
-                            tc_mma_bf16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
-                                             accumulate);
-                        else
-                            tc_mma_bf16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
-                                        accumulate);
+                    for (int h = 0; h < Cfg::NSPLIT; ++h) {
+                        const uint64_t b_desc = smem_desc_sw128(sB + stage * Cfg::B_BYTES +
+                                                                h * Cfg::B_SPLIT_ROWS * 128);
+                        const uint32_t d = d_tmem + h * Cfg::MMA_N;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {  // K = 16 per MMA: +32 bytes in the row
+                            if (kk >= ksteps) break;
+                            const uint32_t accumulate = (kb | kk) != 0;
+                            if constexpr (CG == 2)
+                                tc_mma_bf16_pair(d, a_desc + 2 * kk, b_desc + 2 * kk, idesc,
+                                                 accumulate);
+                            else
+                                tc_mma_bf16(d, a_desc + 2 * kk, b_desc + 2 * kk, idesc, accumulate);
+                        }
                     }
                     if constexpr (CG == 2)
                         tc_commit_pair(empty + stage, kPair);
@@ -452,7 +470,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool resid = args.epi == kEpiResidF32;
         // Single tile per CTA: the residual (x + bias) goes to accumulator 1
         // while the MMAs fill accumulator 0; the drain adds the two.
-        const bool resid_once = resid && args.tma_out && total_tiles <= n_groups;
+        const bool resid_once = Cfg::ACCS == 2 && resid && args.tma_out && total_tiles <= n_groups;
         // Several tiles per CTA: the drain brings each residual piece in by TMA
         // (into the staging box it then stores from) and adds it there.
         const bool resid_drain = resid && args.tma_out && !resid_once;
@@ -708,8 +726,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (resid_once && group < total_tiles) preload(group, 1);
         int it = 0;
         for (int tile = group; tile < total_tiles; tile += n_groups, ++it) {
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
+            const int acc = it % Cfg::ACCS;
+            const uint32_t acc_phase = (uint32_t)(it / Cfg::ACCS) & 1u;
             if (args.tma_out && args.bias && (!resid || resid_drain) && lane * 4 < BN / 2)
                 prefetch_l1(args.bias + (tile % args.num_n_tiles) * BN + half * (BN / 2) + lane * 4);
             if (resid_drain && lane == 0 &&  // first residual piece lands during the mainloop
