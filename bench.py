@@ -45,10 +45,10 @@ UNIT = "audio-s/s"
 # fc2; 4 launches per layer).  DRAM bytes (read + write) per launch, mean over
 # layer 0's four launches of one omni_16req forward (every layer has the same
 # shapes), from one ncu capture of the current kernel: dram__bytes_read.sum +
-# dram__bytes_write.sum of 18.26 / 28.34 / 21.54 / 63.31 MB (the command and
+# dram__bytes_write.sum of 18.26 / 28.34 / 21.57 / 63.51 MB (the command and
 # the table are in profiles/gemm_tc_kernel_dram_omni_16req.md).  Set to None
 # whenever the kernel changes.
-LAYER_GEMM_DRAM_BYTES_PER_LAUNCH = 32.863e6
+LAYER_GEMM_DRAM_BYTES_PER_LAUNCH = 32.920e6
 LAYER_GEMMS = ("qkv", "o_proj", "fc1", "fc2")
 
 
