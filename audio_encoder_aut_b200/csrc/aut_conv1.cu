@@ -14,21 +14,25 @@
 // (row 0 and column 0 are conv2's zero padding).  One tile is 5 plane rows x
 // 25 columns of one plane of one chunk (125 positions in M = 128 rows; the
 // last tile of a plane has 2 rows), so its output is one TMA store box per
-// 64-channel block, [64 channels, 25 columns, 5 rows], straight into the plane.
+// 32-channel block, [32 channels, 25 columns, 5 rows], straight into the plane.
 //
-// Block = 12 warps:
+// The accumulator is split in two halves, channels [0, 256) and [256, C), each
+// its own MMA (N <= 256) with its own full/empty barriers, so the next tile's
+// first half is computed while the epilogue still drains this tile's second.
+//
+// Block = 20 warps:
 //   warp 0     writes each tile's A operand (9 taps per row, 128-byte swizzle)
 //              into one of two buffers, from the chunk's mel tile
-//   warps 10-11  stage the CTA's chunks' mel tiles in shared memory (zero
+//   warps 18-19  stage the CTA's chunks' mel tiles in shared memory (zero
 //              outside the mel bins and past the request's valid frames), two
 //              buffers, many loads in flight per lane
-//   warp 1     allocates tensor memory and issues the tile's two MMAs
-//              (N = C / 2 each) from one thread
-//   warps 2-9  epilogue: two groups of four warps (one per TMEM lane quadrant)
-//              take alternate 64-channel blocks; per block, bias + GELU to
-//              bf16 into a swizzled staging box, then one TMA store.  They also
-//              write the zero borders of both plane sets for the chunks whose
-//              first tile their CTA owns.
+//   warp 1     allocates tensor memory and issues the tile's MMAs (one per
+//              accumulator half) from one thread
+//   warps 2-17 epilogue: four groups of four warps (one per TMEM lane
+//              quadrant) take every fourth 32-channel block; per block, GELU
+//              to bf16 into a 64-byte-swizzled staging box, then one TMA
+//              store.  They also write the zero borders of both plane sets
+//              for the chunks whose first tile their CTA owns.
 // Tiles are split into contiguous ranges, one per CTA (a CTA meets at most a
 // few chunks).  Every mbarrier wait is bounded; on time-out the kernel records
 // AUT_ERR_TIMEOUT and stops.
@@ -54,13 +58,17 @@ constexpr int kPlaneCols = kP1Cols - 1;                               // 25 outp
 constexpr int kMelRowsPad = kMelBins + 2;                             // bins -1 .. 128
 constexpr int kMelColsPad = 104;                                      // frames -1 .. 102
 constexpr int kMaxC = 512;
-constexpr int kThreadsC1 = 384;
-constexpr int kLoaderWarp0 = 10;  // warps 10 and 11 stage mel tiles
+constexpr int kHalfN = 256;       // accumulator half: channels [0, 256) and [256, C)
+constexpr int kGroups = 4;        // epilogue groups of four warps
+constexpr int kEpiWarps = 4 * kGroups;
+constexpr int kThreadsC1 = 32 * (2 + kEpiWarps + 2);
+constexpr int kLoaderWarp0 = 2 + kEpiWarps;  // the last two warps stage mel tiles
+constexpr int kBoxBytes = 128 * 64;          // 128 positions x 32 channels
 constexpr int kMelBytes = ((kMelRowsPad * kMelColsPad * 2 + 1023) / 1024) * 1024;
 constexpr int kOffB = 0;                                   // C rows x 128 B
 constexpr int kOffA = kOffB + kMaxC * 128;                 // 2 x 16 KB
-constexpr int kOffOut = kOffA + 2 * 16384;                 // 2 groups x 2 boxes x 16 KB
-constexpr int kOffMel = kOffOut + 4 * 16384;               // 2 x bf16 [130][104]
+constexpr int kOffOut = kOffA + 2 * 16384;                 // 4 groups x 2 boxes x 8 KB
+constexpr int kOffMel = kOffOut + kGroups * 2 * kBoxBytes;  // 2 x bf16 [130][104]
 constexpr int kOffBar = kOffMel + 2 * kMelBytes;
 constexpr int kSmemC1 = 1024 + kOffBar + 128;
 
@@ -97,15 +105,16 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
     uint8_t *mel_base = sm + kOffMel;
     uint64_t *a_full = reinterpret_cast<uint64_t *>(sm + kOffBar);  // [2]
     uint64_t *a_empty = a_full + 2;                                  // [2]
-    uint64_t *t_full = a_empty + 2;
-    uint64_t *t_empty = t_full + 1;  // count 8: every epilogue warp has read the accumulator
-    uint64_t *mma_done = t_empty + 1;
+    uint64_t *t_full = a_empty + 2;   // [2] per accumulator half
+    uint64_t *t_empty = t_full + 2;   // [2] count 16: every epilogue warp has read the half
+    uint64_t *mma_done = t_empty + 2;
     uint64_t *mel_full = mma_done + 1;   // [2] count 2: both loader warps have staged the tile
     uint64_t *mel_empty = mel_full + 2;  // [2] the builder is done with the tile
     uint32_t *tslot = reinterpret_cast<uint32_t *>(mel_empty + 2);
     int *abort_flag = reinterpret_cast<int *>(tslot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int half_n = C / 2;
+    const int n0 = C < kHalfN ? C : kHalfN;  // channels in the first accumulator half
+    const int n_half = C > kHalfN ? 2 : 1;
 
     pdl_trigger();
     if (threadIdx.x == 0) {
@@ -113,8 +122,10 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
             mbar_init(a_full + i, 1);
             mbar_init(a_empty + i, 1);
         }
-        mbar_init(t_full, 1);
-        mbar_init(t_empty, 8);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(t_full + i, 1);
+            mbar_init(t_empty + i, kEpiWarps);
+        }
         mbar_init(mma_done, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(mel_full + i, 2);
@@ -258,21 +269,29 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
     } else if (warp == 1) {
         if (lane == 0) {
             // -------------------------------------------------- MMA issuer --
-            const uint32_t idesc = idesc_bf16_f32(128, half_n);
+            // Half h: channels [h * 256, h * 256 + N_h), N_h a multiple of 32.
+            const uint32_t idesc0 = idesc_bf16_f32(128, n0);
+            const uint32_t idesc1 = idesc_bf16_f32(128, n_half > 1 ? C - kHalfN : 32);
             bool ok = true;
-            for (int t = 0; t < n_my; ++t) {
+            for (int t = 0; t < n_my && ok; ++t) {
                 const int buf = t & 1;
-                if (!mbar_wait(a_full + buf, (uint32_t)(t >> 1) & 1u, abort_v, lim) ||
-                    (t > 0 && !mbar_wait(t_empty, (uint32_t)(t - 1) & 1u, abort_v, lim))) {
+                if (!mbar_wait(a_full + buf, (uint32_t)(t >> 1) & 1u, abort_v, lim)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 const uint64_t a_desc = smem_desc_sw128(sA + buf * 16384);
-                tc_mma_bf16(tmem, a_desc, smem_desc_sw128(sB), idesc, 0);
-                tc_mma_bf16(tmem + half_n, a_desc, smem_desc_sw128(sB + half_n * 128), idesc, 0);
-                tc_commit(a_empty + buf);
-                tc_commit(t_full);
+                for (int h = 0; h < n_half; ++h) {
+                    // The epilogue has read this half of the previous tile.
+                    if (t > 0 && !mbar_wait(t_empty + h, (uint32_t)(t - 1) & 1u, abort_v, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    tc_mma_bf16(tmem + h * kHalfN, a_desc, smem_desc_sw128(sB + h * kHalfN * 128),
+                                h ? idesc1 : idesc0, 0);
+                    tc_commit(t_full + h);
+                }
+                if (ok) tc_commit(a_empty + buf);
             }
             if (!ok) c1_abort(status, abort_v);
             tc_commit(mma_done);
@@ -280,15 +299,16 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
         }
     } else {
         // ------------------------------------------------------- epilogue --
-        const int quad = warp & 3, grp = (warp - 2) >> 2;
-        const int row = quad * 32 + lane;  // TMEM lane = position of the tile
+        const int ew = warp - 2;                     // 0 .. 15
+        const int quad = warp & 3, grp = ew >> 2;   // TMEM lane quadrant, group
+        const int row = quad * 32 + lane;            // TMEM lane = position of the tile
         const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16);
-        const bool issuer = warp == 2 + 4 * grp && lane == 0;
-        const int n_blk = (C + 63) / 64;
-        uint8_t *my_out = sOut + grp * 2 * 16384;
-        uint32_t stored = 0;  // boxes this group has stored (warp-uniform)
+        const bool issuer = (ew & 3) == 0 && lane == 0;
+        const int n_blk = C / 32, n_blk0 = n0 / 32;  // 32-channel blocks: all, first half
+        uint8_t *my_out = sOut + grp * 2 * kBoxBytes;
+        uint32_t stored = 0;  // boxes this group has stored (group-uniform)
         bool ok = true;
-        const int gtid = (warp - 2) * 32 + lane;  // 0 .. 255
+        const int gtid = ew * 32 + lane;  // 0 .. 511
         for (int t = 0; t < n_my && ok; ++t) {
             const int gt = t_begin + t, cl = gt / kTilesPerChunk, r = gt - cl * kTilesPerChunk;
             const int plane = r / kBlocksPerPlane, rb = r - plane * kBlocksPerPlane;
@@ -298,7 +318,7 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
                 // column 0 and, in odd-column planes, the missing last column.
                 const int c16 = C / 8;  // 16-byte pieces per pixel
                 const size_t r1 = (size_t)cl * kP1Rows;
-                for (int idx = gtid; idx < 4 * (kP1Cols + kP1Rows - 1) * c16; idx += 256) {
+                for (int idx = gtid; idx < 4 * (kP1Cols + kP1Rows - 1) * c16; idx += 32 * kEpiWarps) {
                     const int pix = idx / c16, q = idx - pix * c16;
                     const int pl = pix / (kP1Cols + kP1Rows - 1), e = pix - pl * (kP1Cols + kP1Rows - 1);
                     const size_t prow = (size_t)pl * plane_rows + r1 + (e < kP1Cols ? 0 : e - kP1Cols + 1);
@@ -308,7 +328,7 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
                 }
                 const size_t r2 = (size_t)cl * kP2Rows;
                 constexpr int kB2 = kP2Cols + 2 * (kP2Rows - 1);  // row 0, column 0, last column
-                for (int idx = gtid; idx < 4 * kB2 * c16; idx += 256) {
+                for (int idx = gtid; idx < 4 * kB2 * c16; idx += 32 * kEpiWarps) {
                     const int pix = idx / c16, q = idx - pix * c16;
                     const int pl = pix / kB2, e = pix - pl * kB2;
                     size_t prow;
@@ -329,51 +349,54 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
                     reinterpret_cast<uint4 *>(planes2 + (prow * kP2Cols + col) * C)[q] = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
-            if (!mbar_wait_warp(t_full, (uint32_t)t & 1u, abort_v, lim)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
             const bool tail = rb == kBlocksPerPlane - 1;
             const bool live = quad * 32 < (tail ? kTailRows : kRowsPerTile) * kPlaneCols;  // warp-uniform
             const int out_row = plane * plane_rows + cl * kP1Rows + 1 + rb * kRowsPerTile;
-            for (int bk = grp; bk < n_blk; bk += 2) {
-                const int c0 = min(64 * bk, C - 64);  // the last block overlaps the one before
-                uint8_t *box = my_out + (stored & 1u) * 16384;
-                // The store issued from this box two blocks ago has read it.
-                if (issuer && stored >= 2) bulk_wait_read_1();
-                bar_named(1 + grp, 128);
-                if (live) {  // a quadrant past the tile's positions is never stored
-                    float v[2][32];
-                    tmem_ld32(t_row + c0, v[0]);
-                    tmem_ld32(t_row + c0 + 32, v[1]);
-                    tc_wait_ld();
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
+            for (int h = 0; h < n_half; ++h) {
+                if (!mbar_wait_warp(t_full + h, (uint32_t)t & 1u, abort_v, lim)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // This group's blocks of the half: every fourth, counted from block 0.
+                const int b_lo = h ? n_blk0 : 0, b_hi = h ? n_blk : n_blk0;
+                for (int bk = b_lo + ((grp - b_lo) & (kGroups - 1)); bk < b_hi; bk += kGroups) {
+                    const int c0 = 32 * bk;
+                    uint8_t *box = my_out + (stored & 1u) * kBoxBytes;
+                    // The store issued from this box two blocks ago has read it.
+                    if (issuer && stored >= 2) bulk_wait_read_1();
+                    bar_named(1 + grp, 128);
+                    if (live) {  // a quadrant past the tile's positions is never stored
+                        float v[32];
+                        tmem_ld32(t_row + c0, v);
+                        tc_wait_ld();
+                        uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 32; j += 2) {
-                            const float2 g = gelu_fast2(make_float2(v[hh][j], v[hh][j + 1]));
-                            pk[16 * hh + j / 2] = pack_bf16x2(g.x, g.y);
+                            const float2 g = gelu_fast2(make_float2(v[j], v[j + 1]));
+                            pk[j / 2] = pack_bf16x2(g.x, g.y);
                         }
-                    uint8_t *rp = box + row * 128;
+                        // 64-byte rows, 64-byte swizzle: the 16-byte chunk j of row m
+                        // sits at chunk j ^ ((m >> 1) & 3).
+                        uint8_t *rp = box + row * 64;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)  // 16-byte chunk j of this row, 128-byte swizzle
-                        *reinterpret_cast<uint4 *>(rp + ((j ^ (row & 7)) << 4)) =
-                            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(rp + ((j ^ ((row >> 1) & 3)) << 4)) =
+                                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    bar_named(1 + grp, 128);
+                    if (issuer) {
+                        tma_store_3d(tail ? &tm_out2 : &tm_out5, box, c0, 1, out_row);
+                        bulk_commit();
+                    }
+                    ++stored;
                 }
-                fence_proxy_async_smem();
-                bar_named(1 + grp, 128);
-                if (issuer) {
-                    tma_store_3d(tail ? &tm_out2 : &tm_out5, box, c0, 1, out_row);
-                    bulk_commit();
-                }
-                ++stored;
+                // Every TMEM read of this half is done: the next tile's MMA may write it.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(t_empty + h);
             }
-            // Every TMEM read of this tile is done: the next tile's MMAs may write.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(t_empty);
         }
         if (!ok && lane == 0) c1_abort(status, abort_v);
         if (issuer) bulk_wait_read_all();  // the staged boxes are read before the block exits
@@ -400,14 +423,14 @@ cudaError_t launch_conv1_tc(const void *feats, int T_max, const int4 *chunks, in
     const cudaError_t e = smem_attr_once<conv1_tc_kernel>(kSmemC1);
     if (e != cudaSuccess) return e;
     // conv2's input planes as [4 * plane_rows rows][kP1Cols columns][C]: boxes of
-    // 64 channels x 25 columns x 5 (or 2) rows.
+    // 32 channels x 25 columns x 5 (or 2) rows, 64-byte swizzle.
     CUtensorMap tm5, tm2;
     const uint64_t dims[3] = {(uint64_t)C, (uint64_t)kP1Cols, (uint64_t)4 * plane_rows};
     const uint64_t strides[2] = {(uint64_t)C * 2, (uint64_t)kP1Cols * C * 2};
-    const uint32_t box5[3] = {64, (uint32_t)kPlaneCols, (uint32_t)kRowsPerTile};
-    const uint32_t box2[3] = {64, (uint32_t)kPlaneCols, (uint32_t)kTailRows};
-    if (!make_tensor_map_bf16_sw128(&tm5, 3, planes, dims, strides, box5) ||
-        !make_tensor_map_bf16_sw128(&tm2, 3, planes, dims, strides, box2))
+    const uint32_t box5[3] = {32, (uint32_t)kPlaneCols, (uint32_t)kRowsPerTile};
+    const uint32_t box2[3] = {32, (uint32_t)kPlaneCols, (uint32_t)kTailRows};
+    if (!make_tensor_map_bf16_sw64(&tm5, 3, planes, dims, strides, box5) ||
+        !make_tensor_map_bf16_sw64(&tm2, 3, planes, dims, strides, box2))
         return cudaErrorInvalidValue;
     const int tiles = n_chunks * kTilesPerChunk;
     const int grid = std::min(tiles, sm_count_cached());

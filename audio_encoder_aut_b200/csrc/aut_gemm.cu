@@ -32,23 +32,24 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle; dims innermost first, strides in bytes
-// for dims 1.., box in elements.  Out-of-range elements of a box read as zero.
+// bf16 tensor map (128-byte swizzle unless asked otherwise); dims innermost
+// first, strides in bytes for dims 1.., box in elements.  Out-of-range elements
+// of a box read as zero.
 bool make_map(CUtensorMap *m, int rank, const void *ptr, const cuuint64_t *dims,
               const cuuint64_t *strides, const cuuint32_t *box,
-              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
     return fn(m, dtype, (cuuint32_t)rank, const_cast<void *>(ptr), dims,
-              strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
-                                const uint64_t *strides, const uint32_t *box) {
+bool make_map_bf16(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
+                   const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swizzle) {
+    if (rank < 1 || rank > 5) return false;
     cuuint64_t dd[5], ss[4];
     cuuint32_t bb[5];
     for (int i = 0; i < rank; ++i) {
@@ -56,7 +57,19 @@ bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const
         bb[i] = box[i];
         if (i + 1 < rank) ss[i] = strides[i];
     }
-    return make_map(m, rank, ptr, dd, ss, bb);
+    return make_map(m, rank, ptr, dd, ss, bb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, swizzle);
+}
+
+}  // namespace
+
+bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
+                                const uint64_t *strides, const uint32_t *box) {
+    return make_map_bf16(m, rank, ptr, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool make_tensor_map_bf16_sw64(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
+                               const uint64_t *strides, const uint32_t *box) {
+    return make_map_bf16(m, rank, ptr, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 namespace {

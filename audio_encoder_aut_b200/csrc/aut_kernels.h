@@ -121,6 +121,10 @@ cudaError_t launch_window_attention_tc(const void *qkv, void *out, const int *cu
 // strides in bytes for dims 1.., box in elements.
 bool make_tensor_map_bf16_sw128(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
                                 const uint64_t *strides, const uint32_t *box);
+// The same with 64-byte swizzle (an inner box of at most 64 bytes): the 16-byte
+// chunk c of a box row at shared address a sits at chunk c ^ ((a >> 7) & 3).
+bool make_tensor_map_bf16_sw64(CUtensorMap *m, int rank, const void *ptr, const uint64_t *dims,
+                               const uint64_t *strides, const uint32_t *box);
 cudaError_t launch_prepare(const void *conv2_w, const void *conv3_w, const void *conv_out_w,
                            void *conv2_tap, void *conv3_tap, void *conv_out_fc, float *pos, int C,
                            int d, cudaStream_t st);
