@@ -111,10 +111,11 @@ def test_asr06b_nonlinear_stem():
 
 @pytest.mark.parametrize("C", [64, 192, 240, 256, 384, 512])
 def test_stem_channel_counts(C):
-    """The stem at other conv widths: C = 64 .. 512 on the tensor-core conv1
-    (one or two blocks per group, no overlap or an overlapping last block,
-    N = C / 2 per MMA up to 256), C = 240 on the CUDA-core conv1; partial last
-    chunks; GELUs in their non-linear range (conv weights x 25)."""
+    """The stem at other supported conv widths: C = 64 .. 512 on the tensor-core
+    conv1 (accumulator halves of N = min(C, 256) and C - 256: one half up to
+    C = 256, two from 384; epilogue groups without a block at C = 64), C = 240
+    on the CUDA-core conv1; partial last chunks; GELUs in their non-linear range
+    (conv weights x 25)."""
     import dataclasses
     cfg = dataclasses.replace(S.TINY, downsample_hidden_size=C)
     w = S.weights(cfg, conv_scale=25.0)
