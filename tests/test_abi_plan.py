@@ -82,6 +82,17 @@ def test_workspace_and_prepared_sizes():
     assert A.aut_workspace_bytes(bad, 10, 1, 1) == 0
 
 
+def test_conv_widths_accepted_are_the_documented_set():
+    """aut.h documents conv_ch as one of 16, 32, 64, 128, 192, 240, 256, 384,
+    480, 512; every other width up to 1024 is refused before any launch."""
+    documented = {16, 32, 64, 128, 192, 240, 256, 384, 480, 512}
+    for C in range(1, 1025):
+        c = A.make_config(S.OMNI)
+        c.conv_ch = C
+        assert (A.aut_prepared_bytes(c) > 0) == (C in documented), C
+        assert (A.aut_plan_status(c, [100]) == A.AUT_OK) == (C in documented), C
+
+
 def test_entry_points_reject_before_launch():
     """Argument errors come back without touching a GPU (none is present here)."""
     L = A.lib()
