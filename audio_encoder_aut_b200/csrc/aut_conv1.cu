@@ -74,6 +74,11 @@ constexpr int kSmemC1 = 1024 + kOffBar + 128;
 
 static_assert(kP1Rows - 1 == 32 && kPlaneCols == 25, "conv1 output 64 x 50");
 static_assert(kRowsPerTile * kPlaneCols <= 128, "a tile fits M = 128");
+static_assert(kSmemC1 <= 227 * 1024, "shared memory of one CTA");
+static_assert(kThreadsC1 <= 1024 && kEpiWarps % 4 == 0, "whole lane quadrants per group");
+static_assert(kBoxBytes % 512 == 0 && kOffOut % 1024 == 0, "64-byte swizzle boxes on 512-byte atoms");
+static_assert(kOffA % 1024 == 0 && kOffMel % 16 == 0, "128-byte swizzle operands on 1024-byte atoms");
+static_assert((kGroups & (kGroups - 1)) == 0, "groups take blocks by a power-of-two stride");
 
 AUT_DEV void bar_named(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
