@@ -312,12 +312,16 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
         const int n_blk = C / 32, n_blk0 = n0 / 32;  // 32-channel blocks: all, first half
         uint8_t *my_out = sOut + grp * 2 * kBoxBytes;
         uint32_t stored = 0;  // boxes this group has stored (group-uniform)
+        // Warp-uniform; false once a wait of this warp has given up.  A warp that
+        // gives up raises the abort and then still walks every remaining block
+        // with its group, skipping its waits, TMEM loads and stores, so that no
+        // warp of the group is left at a group barrier (which has no time limit).
         bool ok = true;
         const int gtid = ew * 32 + lane;  // 0 .. 511
-        for (int t = 0; t < n_my && ok; ++t) {
+        for (int t = 0; t < n_my; ++t) {
             const int gt = t_begin + t, cl = gt / kTilesPerChunk, r = gt - cl * kTilesPerChunk;
             const int plane = r / kBlocksPerPlane, rb = r - plane * kBlocksPerPlane;
-            if (r == 0) {
+            if (r == 0 && ok) {
                 // This chunk's zero borders: row 0 and column 0 of its four conv2
                 // input planes, and of conv3's input planes (conv2's output) row 0,
                 // column 0 and, in odd-column planes, the missing last column.
@@ -358,9 +362,9 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
             const bool live = quad * 32 < (tail ? kTailRows : kRowsPerTile) * kPlaneCols;  // warp-uniform
             const int out_row = plane * plane_rows + cl * kP1Rows + 1 + rb * kRowsPerTile;
             for (int h = 0; h < n_half; ++h) {
-                if (!mbar_wait_warp(t_full + h, (uint32_t)t & 1u, abort_v, lim)) {
+                if (ok && !mbar_wait_warp(t_full + h, (uint32_t)t & 1u, abort_v, lim)) {
                     ok = false;
-                    break;
+                    if (lane == 0) c1_abort(status, abort_v);
                 }
                 tc_fence_after();
                 // This group's blocks of the half: every fourth, counted from block 0.
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
                     // The store issued from this box two blocks ago has read it.
                     if (issuer && stored >= 2) bulk_wait_read_1();
                     bar_named(1 + grp, 128);
-                    if (live) {  // a quadrant past the tile's positions is never stored
+                    if (live && ok) {  // a quadrant past the tile's positions is never stored
                         float v[32];
                         tmem_ld32(t_row + c0, v);
                         tc_wait_ld();
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
                     }
                     fence_proxy_async_smem();
                     bar_named(1 + grp, 128);
-                    if (issuer) {
+                    if (issuer && ok) {
                         tma_store_3d(tail ? &tm_out2 : &tm_out5, box, c0, 1, out_row);
                         bulk_commit();
                     }
@@ -403,7 +407,6 @@ __global__ void __launch_bounds__(kThreadsC1, 1) conv1_tc_kernel(
                 if (lane == 0) mbar_arrive(t_empty + h);
             }
         }
-        if (!ok && lane == 0) c1_abort(status, abort_v);
         if (issuer) bulk_wait_read_all();  // the staged boxes are read before the block exits
     }
     tc_fence_before();
